@@ -1,0 +1,212 @@
+"""CPU oracle of the error-bounded lossy encoding -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference
+legs of ``bench.py`` may import this package.  The product library
+(``error_bounded_lossy_encode_b200``) never imports it and shares no code with
+it: the oracle is plain scalar C (``eblc_oracle.c``) built with gcc, wrapped
+here with ctypes and numpy for marshalling only.
+
+What each function computes, with its source (page title, section), is stated
+in ``eblc_oracle.c``.  Every function here has at least one pin in
+``tests/test_oracle_pins.py`` that checks it against something other than
+itself (exact rational arithmetic, library routines, closed forms, a
+hand-derived worked example, brute force over tiny inputs).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "eblc_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+ERR_ARG, ERR_CAPACITY, ERR_OUTLIER_CAP, ERR_CORRUPT, ERR_NOMEM = -1, -2, -3, -4, -5
+CHUNK = 4096
+HEADER_BYTES = 128
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with IEEE semantics (no FMA contraction, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+               "-fPIC", "-shared", "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+class _Header(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_uint32) for k in ("magic", "version", "flags", "block", "chunk", "pad")] + \
+               [(k, ctypes.c_uint64) for k in ("n", "nb", "nc", "W", "m", "total")] + \
+               [("eb", ctypes.c_double), ("bound", ctypes.c_double)] + \
+               [(k, ctypes.c_float) for k in ("inv2eb", "step", "vmin", "vmax")] + \
+               [(k, ctypes.c_uint64) for k in ("width_off", "index_off", "payload_off", "idx_off", "val_off")]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        u64, u32, i32, dbl, flt = ctypes.c_uint64, ctypes.c_uint32, ctypes.c_int32, ctypes.c_double, ctypes.c_float
+        L.orc_value_range.argtypes = [P, u64, P, P]
+        L.orc_value_range.restype = ctypes.c_int
+        L.orc_resolve_bound.argtypes = [ctypes.c_int, dbl, flt, flt, P, P, P]
+        L.orc_resolve_bound.restype = None
+        L.orc_quantize.argtypes = [P, u64, flt, flt, dbl, P, P]
+        L.orc_quantize.restype = None
+        L.orc_zigzag.argtypes = [i32]
+        L.orc_zigzag.restype = u32
+        L.orc_unzigzag.argtypes = [u32]
+        L.orc_unzigzag.restype = i32
+        L.orc_block_width.argtypes = [P, u32]
+        L.orc_block_width.restype = u32
+        L.orc_block_words.argtypes = [u32, u32]
+        L.orc_block_words.restype = u32
+        L.orc_pack_block.argtypes = [P, u32, u32, P]
+        L.orc_pack_block.restype = None
+        L.orc_unpack_block.argtypes = [P, u32, u32, P]
+        L.orc_unpack_block.restype = None
+        L.orc_max_compressed_bytes.argtypes = [u64, u32, u64]
+        L.orc_max_compressed_bytes.restype = u64
+        L.orc_compress.argtypes = [P, u64, u32, ctypes.c_int, dbl, u64, P, u64]
+        L.orc_compress.restype = ctypes.c_int64
+        L.orc_parse_header.argtypes = [P, u64, ctypes.POINTER(_Header)]
+        L.orc_parse_header.restype = ctypes.c_int
+        L.orc_decompress.argtypes = [P, u64, P, u64]
+        L.orc_decompress.restype = ctypes.c_int
+        L.orc_block_codes.argtypes = [P, u64, u32, flt, P, P]
+        L.orc_block_codes.restype = None
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def _f32(x) -> np.ndarray:
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def value_range(x):
+    x = _f32(x)
+    lo, hi = np.zeros(1, np.float32), np.zeros(1, np.float32)
+    any_finite = lib().orc_value_range(_ptr(x), x.size, _ptr(lo), _ptr(hi))
+    return float(lo[0]), float(hi[0]), bool(any_finite)
+
+
+@dataclass
+class Bound:
+    eb: float
+    inv2eb: np.float32
+    step: np.float32
+
+
+def resolve_bound(abs_mode: bool, bound: float, vmin: float = 0.0, vmax: float = 0.0) -> Bound:
+    eb, inv, st = np.zeros(1, np.float64), np.zeros(1, np.float32), np.zeros(1, np.float32)
+    lib().orc_resolve_bound(int(abs_mode), float(bound), float(np.float32(vmin)), float(np.float32(vmax)),
+                            _ptr(eb), _ptr(inv), _ptr(st))
+    return Bound(float(eb[0]), inv[0], st[0])
+
+
+def quantize(x, bnd: Bound):
+    x = _f32(x)
+    q = np.zeros(x.size, np.int32)
+    flag = np.zeros(x.size, np.uint8)
+    lib().orc_quantize(_ptr(x), x.size, float(bnd.inv2eb), float(bnd.step), float(bnd.eb), _ptr(q), _ptr(flag))
+    return q, flag.astype(bool)
+
+
+def zigzag(d: int) -> int:
+    return int(lib().orc_zigzag(int(d)))
+
+
+def unzigzag(z: int) -> int:
+    return int(lib().orc_unzigzag(int(z)))
+
+
+def block_width(z) -> int:
+    z = np.ascontiguousarray(z, dtype=np.uint32)
+    return int(lib().orc_block_width(_ptr(z), z.size))
+
+
+def block_words(w: int, cnt: int) -> int:
+    return int(lib().orc_block_words(w, cnt))
+
+
+def pack_block(z, w: int) -> np.ndarray:
+    z = np.ascontiguousarray(z, dtype=np.uint32)
+    out = np.zeros(max(1, block_words(w, z.size)), np.uint32)
+    lib().orc_pack_block(_ptr(z), z.size, w, _ptr(out))
+    return out[: block_words(w, z.size)]
+
+
+def unpack_block(words, cnt: int, w: int) -> np.ndarray:
+    words = np.ascontiguousarray(words, dtype=np.uint32)
+    if words.size == 0:
+        words = np.zeros(1, np.uint32)
+    z = np.zeros(max(1, cnt), np.uint32)
+    lib().orc_unpack_block(_ptr(words), cnt, w, _ptr(z))
+    return z[:cnt]
+
+
+def max_compressed_bytes(n: int, block: int, outlier_cap: int | None = None) -> int:
+    return int(lib().orc_max_compressed_bytes(n, block, n if outlier_cap is None else outlier_cap))
+
+
+def compress(x, block: int = 128, *, rel: float | None = None, abs: float | None = None,
+             outlier_cap: int | None = None, out_cap: int | None = None):
+    """Return the stream as a uint8 array, or raise OracleError(code)."""
+    x = _f32(x).reshape(-1)
+    if (rel is None) == (abs is None):
+        raise ValueError("exactly one of rel / abs")
+    abs_mode = abs is not None
+    bound = float(abs if abs_mode else rel)
+    cap = x.size if outlier_cap is None else int(outlier_cap)
+    need = max_compressed_bytes(x.size, block, cap) if out_cap is None else int(out_cap)
+    out = np.zeros(max(need, 1), np.uint8)
+    rc = lib().orc_compress(_ptr(x), x.size, block, int(abs_mode), bound, cap, _ptr(out), need)
+    if rc < 0:
+        raise OracleError(int(rc))
+    return out[:rc].copy()
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code: int):
+        super().__init__(f"oracle error {code}")
+        self.code = code
+
+
+def parse_header(stream) -> dict:
+    s = np.ascontiguousarray(stream, dtype=np.uint8)
+    h = _Header()
+    rc = lib().orc_parse_header(_ptr(s) if s.size else 0, s.size, ctypes.byref(h))
+    if rc != 0:
+        raise OracleError(rc)
+    return {k: getattr(h, k) for k, _ in _Header._fields_}
+
+
+def decompress(stream, n: int) -> np.ndarray:
+    s = np.ascontiguousarray(stream, dtype=np.uint8)
+    out = np.zeros(max(n, 1), np.float32)
+    rc = lib().orc_decompress(_ptr(s), s.size, _ptr(out), n)
+    if rc != 0:
+        raise OracleError(rc)
+    return out[:n]
+
+
+def block_codes(x, block: int, inv2eb) -> tuple[np.ndarray, np.ndarray]:
+    x = _f32(x).reshape(-1)
+    nb = (x.size + block - 1) // block
+    z = np.zeros(max(1, x.size), np.uint32)
+    w = np.zeros(max(1, nb), np.uint8)
+    lib().orc_block_codes(_ptr(x), x.size, block, float(np.float32(inv2eb)), _ptr(z), _ptr(w))
+    return z[: x.size], w[:nb]

@@ -1,0 +1,493 @@
+/*
+ * eblc_oracle.c -- plain, slow, scalar CPU oracle of the error-bounded lossy
+ * encoding (linear quantizer -> 1-D Lorenzo predictor reset per block ->
+ * zigzag -> adaptive fixed-length bitpack, with an outlier side list and a
+ * cross-block scan/pack into one archive), and of its exact inverse.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the package smoke check and
+ * the CPU-baseline leg of the benchmark load this library.  The product (the
+ * CUDA library) never includes, links or calls anything in this directory, and
+ * this file includes nothing of the product: every constant and layout rule
+ * below is written out here on its own.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared
+ * (no FMA contraction, IEEE single/double arithmetic, round-to-nearest-even).
+ *
+ * Sources (page title, section):
+ *   [SPEC]  FZGPUModules "Pipeline specialization internals":
+ *           "Roles and strategies" (Elementwise linear quantizer, RegionLocal
+ *           1-D Lorenzo with region reset, SegmentCodec adaptive bitpack,
+ *           WarpRegister block = 32*EPL elements);
+ *           "Forward declaration" (block_size % 32 == 0, block = 32*EPL, the
+ *           float inv2eb slot; the quantizer quantizes inline in delta());
+ *           "Inverse declaration" (dequant step = 2*abs_eb; plain
+ *           first-difference undelta);
+ *           "Priming: the fused runner bypasses execute()" (value-range scan
+ *           and bound resolution before the fused kernel; default bound 1e-4;
+ *           the inverse must read the resolved bound);
+ *           "The device policy contract" (coder meta_bytes = 1 per block;
+ *           decode(meta, base, count, ...); Zigzag as an interior transform);
+ *           "Validation requirements" (byte-identical archives, partial final
+ *           block).
+ *   [NVRTC] "nvrtc_chunk_fusion.h File Reference": launchNvrtcChunkFusedEncode
+ *           and launchGenericChunkFusion (split-outlier side output: uint32
+ *           index array + value array with an append counter; cross-chunk
+ *           scan/pack tail returning the archive byte length).
+ *   [DEVITO] "DevitoComp provider interface": "Configuring the error
+ *           tolerance" (non-negative relative error fixed at plan creation).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - relative error is relative to the value range (max - min) over the
+ *     finite elements; with no finite element the range is 0;
+ *   - y = x * inv2eb in float, q = round-half-even(y) when |y| < 2^30, else 0;
+ *   - outlier test: x non-finite, or fp64 |x - x'| > eb, x' = (float)q * step;
+ *     the code q stays in the stream even for an outlier;
+ *   - zigzag is the textbook map d >= 0 -> 2d, d < 0 -> -2d - 1;
+ *   - width = bit length of the OR of the block's zigzag codes (0..32), one
+ *     byte per block; the payload of a block is ceil(w*cnt/32) little-endian
+ *     u32 words holding code j at bits [j*w, j*w + w), least significant first;
+ *   - the partial final block holds only its cnt real elements;
+ *   - outliers are stored sorted by index, value as raw float32 bits.
+ *
+ * Stream layout, version 1 (all little-endian):
+ *   header, 128 bytes:
+ *     0 u32 magic 0x434C4245 ("EBLC")   4 u16 version = 1   6 u16 flags
+ *     (bit0: absolute bound)            8 u64 n             16 u32 block B
+ *     20 u32 chunk = 4096               24 f64 eb           32 f32 inv2eb
+ *     36 f32 step                       40 f32 vmin         44 f32 vmax
+ *     48 u64 nb (blocks)                56 u64 nc (chunks)  64 u64 W (payload
+ *     words)                            72 u64 m (outliers) 80 u64 total bytes
+ *     88 f64 bound as requested (relative or absolute)      96..127 zero
+ *   128:          u8 width[nb], zero padded to a multiple of 16 bytes
+ *   I0:           per chunk c of 4096 elements, u32 pair (word offset of the
+ *                 chunk's first block, number of outliers before the chunk's
+ *                 first element), zero padded to 16
+ *   P0:           payload u32[W], blocks in order, zero padded to 16
+ *   X0:           u32 idx[m] ascending, zero padded to 16
+ *   V0:           u32 val[m] (float32 bits);  total = V0 + 4m.
+ */
+#include <fenv.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_MAGIC 0x434C4245u
+#define ORC_VERSION 1u
+#define ORC_CHUNK 4096u
+#define ORC_HEADER_BYTES 128u
+#define ORC_FLAG_ABS 1u
+
+/* error codes returned as negative values */
+#define ORC_ERR_ARG (-1)
+#define ORC_ERR_CAPACITY (-2)     /* output buffer too small               */
+#define ORC_ERR_OUTLIER_CAP (-3)  /* more outliers than the stated capacity */
+#define ORC_ERR_CORRUPT (-4)
+#define ORC_ERR_NOMEM (-5)
+
+static uint64_t pad16(uint64_t v) { return (v + 15u) / 16u * 16u; }
+
+static void put_u16(uint8_t *p, uint16_t v) { p[0] = (uint8_t)v; p[1] = (uint8_t)(v >> 8); }
+static void put_u32(uint8_t *p, uint32_t v) {
+    for (int i = 0; i < 4; ++i) p[i] = (uint8_t)(v >> (8 * i));
+}
+static void put_u64(uint8_t *p, uint64_t v) {
+    for (int i = 0; i < 8; ++i) p[i] = (uint8_t)(v >> (8 * i));
+}
+static void put_f32(uint8_t *p, float v) { uint32_t u; memcpy(&u, &v, 4); put_u32(p, u); }
+static void put_f64(uint8_t *p, double v) { uint64_t u; memcpy(&u, &v, 8); put_u64(p, u); }
+static uint16_t get_u16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); }
+static uint32_t get_u32(const uint8_t *p) {
+    uint32_t v = 0;
+    for (int i = 3; i >= 0; --i) v = (v << 8) | p[i];
+    return v;
+}
+static uint64_t get_u64(const uint8_t *p) {
+    uint64_t v = 0;
+    for (int i = 7; i >= 0; --i) v = (v << 8) | p[i];
+    return v;
+}
+static float get_f32(const uint8_t *p) { uint32_t u = get_u32(p); float v; memcpy(&v, &u, 4); return v; }
+static double get_f64(const uint8_t *p) { uint64_t u = get_u64(p); double v; memcpy(&v, &u, 8); return v; }
+
+/* ------------------------------------------------------------------------ */
+/* Step 1. Value range over the finite elements ([SPEC] Priming: the
+ * quantizer's value-range scan).  Sequential min/max; each end is then
+ * canonicalised with "+ 0.0f" so that -0.0 reads as +0.0.  Returns 1 if any
+ * element is finite, else 0 (and the range is [0, 0]).                      */
+int orc_value_range(const float *x, uint64_t n, float *vmin_out, float *vmax_out) {
+    int any = 0;
+    float lo = 0.0f, hi = 0.0f;
+    for (uint64_t i = 0; i < n; ++i) {
+        float v = x[i];
+        if (!isfinite(v)) continue;
+        if (!any) {
+            lo = v;
+            hi = v;
+            any = 1;
+        } else {
+            if (v < lo) lo = v;
+            if (v > hi) hi = v;
+        }
+    }
+    *vmin_out = lo + 0.0f;
+    *vmax_out = hi + 0.0f;
+    return any;
+}
+
+/* Step 2. Bound resolution ([SPEC] Priming; Inverse declaration: dequant step
+ * 2*abs_eb; Forward declaration: the float inv2eb slot).  All in IEEE double,
+ * round to nearest, then rounded once to float.                             */
+void orc_resolve_bound(int abs_mode, double bound, float vmin, float vmax,
+                       double *eb_out, float *inv2eb_out, float *step_out) {
+    double eb;
+    if (abs_mode)
+        eb = bound;
+    else
+        eb = bound * ((double)vmax - (double)vmin);
+    double two_eb = 2.0 * eb;
+    double inv = (two_eb == 0.0) ? INFINITY : 1.0 / two_eb;
+    *eb_out = eb;
+    *inv2eb_out = (float)inv;
+    *step_out = (float)two_eb;
+}
+
+/* Step 3. Linear quantization of one element ([SPEC] Roles and strategies:
+ * the linear quantizer is Elementwise, absorbed into the predictor).        */
+static int32_t quant_code(float x, float inv2eb) {
+    float y = x * inv2eb;
+    if (!(fabsf(y) < 1073741824.0f)) /* 2^30; false for NaN and +-Inf */
+        return 0;
+    return (int32_t)nearbyintf(y); /* round half to even (FE_TONEAREST) */
+}
+
+static float dequant(int32_t q, float step) { return (float)q * step; }
+
+/* Outlier test for one element ([NVRTC] split-outlier side output).        */
+static int outlier_test(float x, float xr, double eb) {
+    if (!isfinite(x)) return 1;
+    return !(fabs((double)x - (double)xr) <= eb);
+}
+
+/* Quantize a whole array; exposed so the tests can pin step 3 alone.        */
+void orc_quantize(const float *x, uint64_t n, float inv2eb, float step, double eb,
+                  int32_t *q_out, uint8_t *outlier_out) {
+    for (uint64_t i = 0; i < n; ++i) {
+        int32_t q = quant_code(x[i], inv2eb);
+        q_out[i] = q;
+        outlier_out[i] = (uint8_t)outlier_test(x[i], dequant(q, step), eb);
+    }
+}
+
+/* Step 5. Zigzag (textbook): d >= 0 -> 2d, d < 0 -> -2d - 1.                */
+uint32_t orc_zigzag(int32_t d) {
+    int64_t v = d;
+    if (v >= 0) return (uint32_t)(2 * v);
+    return (uint32_t)(-2 * v - 1);
+}
+
+int32_t orc_unzigzag(uint32_t z) {
+    if ((z & 1u) == 0) return (int32_t)(z / 2u);
+    return (int32_t)(-(int64_t)(z / 2u) - 1);
+}
+
+/* Step 6a. Block width: bit length of the OR of the codes (0..32).          */
+uint32_t orc_block_width(const uint32_t *z, uint32_t cnt) {
+    uint32_t acc = 0, w = 0;
+    for (uint32_t j = 0; j < cnt; ++j) acc |= z[j];
+    while (acc != 0) {
+        ++w;
+        acc >>= 1;
+    }
+    return w;
+}
+
+uint32_t orc_block_words(uint32_t w, uint32_t cnt) {
+    return (uint32_t)(((uint64_t)w * cnt + 31u) / 32u);
+}
+
+/* Step 6b. Fixed-length pack: code j at bits [j*w, j*w+w) of the block's
+ * word array, least significant bit first.  words[] must hold
+ * orc_block_words(w, cnt) words; it is cleared here.                        */
+void orc_pack_block(const uint32_t *z, uint32_t cnt, uint32_t w, uint32_t *words) {
+    uint32_t nw = orc_block_words(w, cnt);
+    for (uint32_t k = 0; k < nw; ++k) words[k] = 0;
+    if (w == 0) return;
+    for (uint32_t j = 0; j < cnt; ++j) {
+        uint64_t pos = (uint64_t)j * w;
+        uint64_t k = pos / 32u;
+        uint32_t sh = (uint32_t)(pos % 32u);
+        uint64_t v = (uint64_t)z[j] << sh;
+        words[k] |= (uint32_t)v;
+        if ((v >> 32) != 0) words[k + 1] |= (uint32_t)(v >> 32);
+    }
+}
+
+void orc_unpack_block(const uint32_t *words, uint32_t cnt, uint32_t w, uint32_t *z) {
+    uint32_t nw = orc_block_words(w, cnt);
+    uint64_t mask = (w == 32) ? 0xFFFFFFFFull : ((1ull << w) - 1ull);
+    for (uint32_t j = 0; j < cnt; ++j) {
+        if (w == 0) {
+            z[j] = 0;
+            continue;
+        }
+        uint64_t pos = (uint64_t)j * w;
+        uint64_t k = pos / 32u;
+        uint32_t sh = (uint32_t)(pos % 32u);
+        uint64_t v = words[k];
+        if (k + 1 < nw) v |= (uint64_t)words[k + 1] << 32;
+        z[j] = (uint32_t)((v >> sh) & mask);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Section offsets of a stream with nb blocks, nc chunks, W words, m outliers */
+typedef struct {
+    uint64_t width_off, index_off, payload_off, idx_off, val_off, total;
+} orc_layout;
+
+static orc_layout layout_of(uint64_t nb, uint64_t nc, uint64_t W, uint64_t m) {
+    orc_layout L;
+    L.width_off = ORC_HEADER_BYTES;
+    L.index_off = L.width_off + pad16(nb);
+    L.payload_off = L.index_off + pad16(8u * nc);
+    L.idx_off = L.payload_off + pad16(4u * W);
+    L.val_off = L.idx_off + pad16(4u * m);
+    L.total = L.val_off + 4u * m;
+    return L;
+}
+
+static int block_ok(uint32_t b) { return b == 32 || b == 64 || b == 128 || b == 256; }
+
+/* Worst-case stream size: every block at width 32 and outlier_cap outliers. */
+uint64_t orc_max_compressed_bytes(uint64_t n, uint32_t block, uint64_t outlier_cap) {
+    if (!block_ok(block)) return 0;
+    uint64_t nb = (n + block - 1) / block;
+    uint64_t nc = (n + ORC_CHUNK - 1) / ORC_CHUNK;
+    return layout_of(nb, nc, n, outlier_cap).total;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Compress x[0..n) into out[0..out_cap).  Returns the stream length, or a
+ * negative ORC_ERR_* code.  Outliers beyond outlier_cap are an error.       */
+int64_t orc_compress(const float *x, uint64_t n, uint32_t block, int abs_mode, double bound,
+                     uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
+    if (!block_ok(block) || !(bound >= 0.0) || !isfinite(bound)) return ORC_ERR_ARG;
+    if (n >= 0xFFFFFFFFull) return ORC_ERR_ARG; /* indices are u32 */
+    if (fegetround() != FE_TONEAREST) return ORC_ERR_ARG;
+
+    /* steps 1-2 */
+    float vmin = 0.0f, vmax = 0.0f;
+    if (!abs_mode) orc_value_range(x, n, &vmin, &vmax);
+    double eb;
+    float inv2eb, step;
+    orc_resolve_bound(abs_mode, bound, vmin, vmax, &eb, &inv2eb, &step);
+
+    uint64_t nb = (n + block - 1) / block;
+    uint64_t nc = (n + ORC_CHUNK - 1) / ORC_CHUNK;
+
+    /* step 3: codes and outlier flags for every element */
+    int32_t *q = (int32_t *)malloc((n ? n : 1) * sizeof(int32_t));
+    uint8_t *flag = (uint8_t *)malloc(n ? n : 1);
+    uint8_t *width = (uint8_t *)malloc(nb ? nb : 1);
+    uint32_t *block_words = (uint32_t *)malloc((nb ? nb : 1) * sizeof(uint32_t));
+    if (!q || !flag || !width || !block_words) {
+        free(q); free(flag); free(width); free(block_words);
+        return ORC_ERR_NOMEM;
+    }
+    orc_quantize(x, n, inv2eb, step, eb, q, flag);
+
+    uint64_t m = 0;
+    for (uint64_t i = 0; i < n; ++i) m += flag[i];
+
+    /* steps 4-6a: per block delta (reset at the block start), zigzag, width */
+    uint32_t z[256];
+    uint64_t W = 0;
+    for (uint64_t b = 0; b < nb; ++b) {
+        uint64_t first = b * block;
+        uint32_t cnt = (uint32_t)((n - first < block) ? (n - first) : block);
+        int32_t prev = 0; /* Lorenzo predecessor resets to 0 at each block */
+        for (uint32_t j = 0; j < cnt; ++j) {
+            int32_t cur = q[first + j];
+            z[j] = orc_zigzag(cur - prev); /* |q| < 2^30 so no overflow */
+            prev = cur;
+        }
+        width[b] = (uint8_t)orc_block_width(z, cnt);
+        block_words[b] = orc_block_words(width[b], cnt);
+        W += block_words[b];
+    }
+
+    orc_layout L = layout_of(nb, nc, W, m);
+    int64_t status = (int64_t)L.total;
+    if (m > outlier_cap) status = ORC_ERR_OUTLIER_CAP;
+    else if (L.total > out_cap) status = ORC_ERR_CAPACITY;
+    if (status < 0) {
+        free(q); free(flag); free(width); free(block_words);
+        return status;
+    }
+
+    memset(out, 0, L.total);
+    /* header */
+    put_u32(out + 0, ORC_MAGIC);
+    put_u16(out + 4, (uint16_t)ORC_VERSION);
+    put_u16(out + 6, (uint16_t)(abs_mode ? ORC_FLAG_ABS : 0u));
+    put_u64(out + 8, n);
+    put_u32(out + 16, block);
+    put_u32(out + 20, ORC_CHUNK);
+    put_f64(out + 24, eb);
+    put_f32(out + 32, inv2eb);
+    put_f32(out + 36, step);
+    put_f32(out + 40, vmin);
+    put_f32(out + 44, vmax);
+    put_u64(out + 48, nb);
+    put_u64(out + 56, nc);
+    put_u64(out + 64, W);
+    put_u64(out + 72, m);
+    put_u64(out + 80, L.total);
+    put_f64(out + 88, bound);
+
+    /* widths */
+    memcpy(out + L.width_off, width, nb);
+
+    /* step 6b + step 8: pack each block at its scanned word offset; record
+     * the chunk index (word offset, outliers before the chunk).            */
+    uint64_t word_off = 0, outl_before = 0, blocks_per_chunk = ORC_CHUNK / block;
+    uint32_t words[256];
+    for (uint64_t b = 0; b < nb; ++b) {
+        uint64_t first = b * block;
+        uint32_t cnt = (uint32_t)((n - first < block) ? (n - first) : block);
+        if (b % blocks_per_chunk == 0) {
+            uint64_t c = b / blocks_per_chunk;
+            put_u32(out + L.index_off + 8 * c, (uint32_t)word_off);
+            put_u32(out + L.index_off + 8 * c + 4, (uint32_t)outl_before);
+        }
+        int32_t prev = 0;
+        for (uint32_t j = 0; j < cnt; ++j) {
+            int32_t cur = q[first + j];
+            z[j] = orc_zigzag(cur - prev);
+            prev = cur;
+            outl_before += flag[first + j];
+        }
+        orc_pack_block(z, cnt, width[b], words);
+        for (uint32_t k = 0; k < block_words[b]; ++k)
+            put_u32(out + L.payload_off + 4 * (word_off + k), words[k]);
+        word_off += block_words[b];
+    }
+
+    /* step 7: the outlier side list, ascending index, raw float bits */
+    uint64_t k = 0;
+    for (uint64_t i = 0; i < n; ++i) {
+        if (!flag[i]) continue;
+        uint32_t bits;
+        memcpy(&bits, &x[i], 4);
+        put_u32(out + L.idx_off + 4 * k, (uint32_t)i);
+        put_u32(out + L.val_off + 4 * k, bits);
+        ++k;
+    }
+
+    free(q); free(flag); free(width); free(block_words);
+    return (int64_t)L.total;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Parsed header, exposed for the tests.                                     */
+typedef struct {
+    uint32_t magic, version, flags, block, chunk, pad;
+    uint64_t n, nb, nc, W, m, total;
+    double eb, bound;
+    float inv2eb, step, vmin, vmax;
+    uint64_t width_off, index_off, payload_off, idx_off, val_off;
+} orc_header;
+
+int orc_parse_header(const uint8_t *s, uint64_t bytes, orc_header *h) {
+    memset(h, 0, sizeof(*h));
+    if (bytes < ORC_HEADER_BYTES) return ORC_ERR_CORRUPT;
+    h->magic = get_u32(s + 0);
+    h->version = get_u16(s + 4);
+    h->flags = get_u16(s + 6);
+    h->n = get_u64(s + 8);
+    h->block = get_u32(s + 16);
+    h->chunk = get_u32(s + 20);
+    h->eb = get_f64(s + 24);
+    h->inv2eb = get_f32(s + 32);
+    h->step = get_f32(s + 36);
+    h->vmin = get_f32(s + 40);
+    h->vmax = get_f32(s + 44);
+    h->nb = get_u64(s + 48);
+    h->nc = get_u64(s + 56);
+    h->W = get_u64(s + 64);
+    h->m = get_u64(s + 72);
+    h->total = get_u64(s + 80);
+    h->bound = get_f64(s + 88);
+    if (h->magic != ORC_MAGIC || h->version != ORC_VERSION || !block_ok(h->block) ||
+        h->chunk != ORC_CHUNK)
+        return ORC_ERR_CORRUPT;
+    if (h->n >= 0xFFFFFFFFull || h->nb != (h->n + h->block - 1) / h->block ||
+        h->nc != (h->n + ORC_CHUNK - 1) / ORC_CHUNK || h->W > h->n || h->m > h->n)
+        return ORC_ERR_CORRUPT;
+    orc_layout L = layout_of(h->nb, h->nc, h->W, h->m);
+    if (L.total != h->total || h->total > bytes) return ORC_ERR_CORRUPT;
+    h->width_off = L.width_off;
+    h->index_off = L.index_off;
+    h->payload_off = L.payload_off;
+    h->idx_off = L.idx_off;
+    h->val_off = L.val_off;
+    return 0;
+}
+
+/* Inverse ([SPEC] Inverse declaration; device policy contract: decode ->
+ * undelta -> dequant code * 2eb), then the outliers are written back.      */
+int orc_decompress(const uint8_t *s, uint64_t bytes, float *out, uint64_t n_expected) {
+    orc_header h;
+    int rc = orc_parse_header(s, bytes, &h);
+    if (rc != 0) return rc;
+    if (h.n != n_expected) return ORC_ERR_ARG;
+
+    uint32_t words[256], z[256];
+    uint64_t word_off = 0;
+    for (uint64_t b = 0; b < h.nb; ++b) {
+        uint64_t first = b * h.block;
+        uint32_t cnt = (uint32_t)((h.n - first < h.block) ? (h.n - first) : h.block);
+        uint32_t w = s[h.width_off + b];
+        if (w > 32) return ORC_ERR_CORRUPT;
+        uint32_t nw = orc_block_words(w, cnt);
+        if (word_off + nw > h.W) return ORC_ERR_CORRUPT;
+        for (uint32_t k = 0; k < nw; ++k)
+            words[k] = get_u32(s + h.payload_off + 4 * (word_off + k));
+        orc_unpack_block(words, cnt, w, z);
+        int64_t qv = 0; /* undelta: running sum restarting at each block */
+        for (uint32_t j = 0; j < cnt; ++j) {
+            qv += orc_unzigzag(z[j]);
+            int32_t q = (int32_t)(uint32_t)(uint64_t)qv;
+            out[first + j] = dequant(q, h.step);
+        }
+        word_off += nw;
+    }
+    if (word_off != h.W) return ORC_ERR_CORRUPT;
+    for (uint64_t k = 0; k < h.m; ++k) {
+        uint32_t i = get_u32(s + h.idx_off + 4 * k);
+        uint32_t bits = get_u32(s + h.val_off + 4 * k);
+        if (i >= h.n) return ORC_ERR_CORRUPT;
+        memcpy(&out[i], &bits, 4);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block-level view for the tests: widths and per-block zigzag codes of the
+ * whole array under given parameters (no stream assembly).                 */
+void orc_block_codes(const float *x, uint64_t n, uint32_t block, float inv2eb,
+                     uint32_t *z_out, uint8_t *width_out) {
+    uint64_t nb = (n + block - 1) / block;
+    for (uint64_t b = 0; b < nb; ++b) {
+        uint64_t first = b * block;
+        uint32_t cnt = (uint32_t)((n - first < block) ? (n - first) : block);
+        int32_t prev = 0;
+        for (uint32_t j = 0; j < cnt; ++j) {
+            int32_t cur = quant_code(x[first + j], inv2eb);
+            z_out[first + j] = orc_zigzag(cur - prev);
+            prev = cur;
+        }
+        width_out[b] = (uint8_t)orc_block_width(z_out + first, cnt);
+    }
+}
