@@ -44,7 +44,7 @@ class _Header(ctypes.Structure):
                [(k, ctypes.c_uint64) for k in ("n", "nb", "nc", "W", "m", "total")] + \
                [("eb", ctypes.c_double), ("bound", ctypes.c_double)] + \
                [(k, ctypes.c_float) for k in ("inv2eb", "step", "vmin", "vmax")] + \
-               [(k, ctypes.c_uint64) for k in ("width_off", "index_off", "payload_off", "idx_off", "val_off")]
+               [(k, ctypes.c_uint64) for k in ("width_off", "index_off", "record_off")]
 
 
 _lib = None

@@ -47,7 +47,9 @@
  *     byte per block; the payload of a block is ceil(w*cnt/32) little-endian
  *     u32 words holding code j at bits [j*w, j*w + w), least significant first;
  *   - the partial final block holds only its cnt real elements;
- *   - outliers are stored sorted by index, value as raw float32 bits.
+ *   - outliers are stored sorted by index, value as raw float32 bits, each
+ *     in the record of the 4096-element chunk that holds it;
+ *   - at most 2^30 elements per stream (record offsets are 32-bit words).
  *
  * Stream layout, version 1 (all little-endian):
  *   header, 128 bytes:
@@ -58,13 +60,14 @@
  *     48 u64 nb (blocks)                56 u64 nc (chunks)  64 u64 W (payload
  *     words)                            72 u64 m (outliers) 80 u64 total bytes
  *     88 f64 bound as requested (relative or absolute)      96..127 zero
- *   128:          u8 width[nb], zero padded to a multiple of 16 bytes
- *   I0:           per chunk c of 4096 elements, u32 pair (word offset of the
- *                 chunk's first block, number of outliers before the chunk's
- *                 first element), zero padded to 16
- *   P0:           payload u32[W], blocks in order, zero padded to 16
- *   X0:           u32 idx[m] ascending, zero padded to 16
- *   V0:           u32 val[m] (float32 bits);  total = V0 + 4m.
+ *   128:  u8 width[nb], zero padded to a multiple of 16 bytes
+ *   I0:   per chunk c (elements [4096c, 4096c + 4096)), a u32 pair: the word
+ *         offset of the chunk's record from P0, and the number of outliers
+ *         before the chunk's first element; zero padded to 16
+ *   P0:   one record per chunk, in order: the payload words of the chunk's
+ *         blocks, then u32 idx[m_c] (ascending element index), then u32
+ *         val[m_c] (float32 bits) of the chunk's m_c outliers.
+ *   total = P0 + 4 * (W + 2m).
  */
 #include <fenv.h>
 #include <math.h>
@@ -241,23 +244,24 @@ void orc_unpack_block(const uint32_t *words, uint32_t cnt, uint32_t w, uint32_t 
 }
 
 /* ------------------------------------------------------------------------ */
-/* Section offsets of a stream with nb blocks, nc chunks, W words, m outliers */
+/* Section offsets of a stream with nb blocks, nc chunks, W payload words and
+ * m outliers.                                                               */
 typedef struct {
-    uint64_t width_off, index_off, payload_off, idx_off, val_off, total;
+    uint64_t width_off, index_off, record_off, total;
 } orc_layout;
 
 static orc_layout layout_of(uint64_t nb, uint64_t nc, uint64_t W, uint64_t m) {
     orc_layout L;
     L.width_off = ORC_HEADER_BYTES;
     L.index_off = L.width_off + pad16(nb);
-    L.payload_off = L.index_off + pad16(8u * nc);
-    L.idx_off = L.payload_off + pad16(4u * W);
-    L.val_off = L.idx_off + pad16(4u * m);
-    L.total = L.val_off + 4u * m;
+    L.record_off = L.index_off + pad16(8u * nc);
+    L.total = L.record_off + 4u * (W + 2u * m);
     return L;
 }
 
 static int block_ok(uint32_t b) { return b == 32 || b == 64 || b == 128 || b == 256; }
+
+#define ORC_MAX_N (1ull << 30)
 
 /* Worst-case stream size: every block at width 32 and outlier_cap outliers. */
 uint64_t orc_max_compressed_bytes(uint64_t n, uint32_t block, uint64_t outlier_cap) {
@@ -269,11 +273,11 @@ uint64_t orc_max_compressed_bytes(uint64_t n, uint32_t block, uint64_t outlier_c
 
 /* ------------------------------------------------------------------------ */
 /* Compress x[0..n) into out[0..out_cap).  Returns the stream length, or a
- * negative ORC_ERR_* code.  Outliers beyond outlier_cap are an error.       */
+ * negative ORC_ERR_* code.  More outliers than outlier_cap is an error.     */
 int64_t orc_compress(const float *x, uint64_t n, uint32_t block, int abs_mode, double bound,
                      uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
     if (!block_ok(block) || !(bound >= 0.0) || !isfinite(bound)) return ORC_ERR_ARG;
-    if (n >= 0xFFFFFFFFull) return ORC_ERR_ARG; /* indices are u32 */
+    if (n > ORC_MAX_N) return ORC_ERR_ARG;
     if (fegetround() != FE_TONEAREST) return ORC_ERR_ARG;
 
     /* steps 1-2 */
@@ -349,40 +353,45 @@ int64_t orc_compress(const float *x, uint64_t n, uint32_t block, int abs_mode, d
     /* widths */
     memcpy(out + L.width_off, width, nb);
 
-    /* step 6b + step 8: pack each block at its scanned word offset; record
-     * the chunk index (word offset, outliers before the chunk).            */
-    uint64_t word_off = 0, outl_before = 0, blocks_per_chunk = ORC_CHUNK / block;
+    /* step 6b + step 8, chunk by chunk: the chunk index entry (record word
+     * offset, outliers so far), then each block packed at the scanned word
+     * offset, then the chunk's outliers ([NVRTC] split-outlier side output,
+     * index array then value array; step 7).                               */
+    uint64_t rec = 0, outl_before = 0, blocks_per_chunk = ORC_CHUNK / block;
     uint32_t words[256];
-    for (uint64_t b = 0; b < nb; ++b) {
-        uint64_t first = b * block;
-        uint32_t cnt = (uint32_t)((n - first < block) ? (n - first) : block);
-        if (b % blocks_per_chunk == 0) {
-            uint64_t c = b / blocks_per_chunk;
-            put_u32(out + L.index_off + 8 * c, (uint32_t)word_off);
-            put_u32(out + L.index_off + 8 * c + 4, (uint32_t)outl_before);
+    for (uint64_t c = 0; c < nc; ++c) {
+        put_u32(out + L.index_off + 8 * c, (uint32_t)rec);
+        put_u32(out + L.index_off + 8 * c + 4, (uint32_t)outl_before);
+        uint64_t b_end = (c + 1) * blocks_per_chunk < nb ? (c + 1) * blocks_per_chunk : nb;
+        for (uint64_t b = c * blocks_per_chunk; b < b_end; ++b) {
+            uint64_t first = b * block;
+            uint32_t cnt = (uint32_t)((n - first < block) ? (n - first) : block);
+            int32_t prev = 0;
+            for (uint32_t j = 0; j < cnt; ++j) {
+                int32_t cur = q[first + j];
+                z[j] = orc_zigzag(cur - prev);
+                prev = cur;
+            }
+            orc_pack_block(z, cnt, width[b], words);
+            for (uint32_t k = 0; k < block_words[b]; ++k)
+                put_u32(out + L.record_off + 4 * (rec + k), words[k]);
+            rec += block_words[b];
         }
-        int32_t prev = 0;
-        for (uint32_t j = 0; j < cnt; ++j) {
-            int32_t cur = q[first + j];
-            z[j] = orc_zigzag(cur - prev);
-            prev = cur;
-            outl_before += flag[first + j];
+        uint64_t e_first = c * ORC_CHUNK;
+        uint64_t e_end = e_first + ORC_CHUNK < n ? e_first + ORC_CHUNK : n;
+        uint64_t mc = 0;
+        for (uint64_t i = e_first; i < e_end; ++i) mc += flag[i];
+        uint64_t k = 0;
+        for (uint64_t i = e_first; i < e_end; ++i) {
+            if (!flag[i]) continue;
+            uint32_t bits;
+            memcpy(&bits, &x[i], 4);
+            put_u32(out + L.record_off + 4 * (rec + k), (uint32_t)i);
+            put_u32(out + L.record_off + 4 * (rec + mc + k), bits);
+            ++k;
         }
-        orc_pack_block(z, cnt, width[b], words);
-        for (uint32_t k = 0; k < block_words[b]; ++k)
-            put_u32(out + L.payload_off + 4 * (word_off + k), words[k]);
-        word_off += block_words[b];
-    }
-
-    /* step 7: the outlier side list, ascending index, raw float bits */
-    uint64_t k = 0;
-    for (uint64_t i = 0; i < n; ++i) {
-        if (!flag[i]) continue;
-        uint32_t bits;
-        memcpy(&bits, &x[i], 4);
-        put_u32(out + L.idx_off + 4 * k, (uint32_t)i);
-        put_u32(out + L.val_off + 4 * k, bits);
-        ++k;
+        rec += 2 * mc;
+        outl_before += mc;
     }
 
     free(q); free(flag); free(width); free(block_words);
@@ -396,7 +405,7 @@ typedef struct {
     uint64_t n, nb, nc, W, m, total;
     double eb, bound;
     float inv2eb, step, vmin, vmax;
-    uint64_t width_off, index_off, payload_off, idx_off, val_off;
+    uint64_t width_off, index_off, record_off;
 } orc_header;
 
 int orc_parse_header(const uint8_t *s, uint64_t bytes, orc_header *h) {
@@ -422,21 +431,20 @@ int orc_parse_header(const uint8_t *s, uint64_t bytes, orc_header *h) {
     if (h->magic != ORC_MAGIC || h->version != ORC_VERSION || !block_ok(h->block) ||
         h->chunk != ORC_CHUNK)
         return ORC_ERR_CORRUPT;
-    if (h->n >= 0xFFFFFFFFull || h->nb != (h->n + h->block - 1) / h->block ||
+    if (h->n > ORC_MAX_N || h->nb != (h->n + h->block - 1) / h->block ||
         h->nc != (h->n + ORC_CHUNK - 1) / ORC_CHUNK || h->W > h->n || h->m > h->n)
         return ORC_ERR_CORRUPT;
     orc_layout L = layout_of(h->nb, h->nc, h->W, h->m);
     if (L.total != h->total || h->total > bytes) return ORC_ERR_CORRUPT;
     h->width_off = L.width_off;
     h->index_off = L.index_off;
-    h->payload_off = L.payload_off;
-    h->idx_off = L.idx_off;
-    h->val_off = L.val_off;
+    h->record_off = L.record_off;
     return 0;
 }
 
 /* Inverse ([SPEC] Inverse declaration; device policy contract: decode ->
- * undelta -> dequant code * 2eb), then the outliers are written back.      */
+ * undelta -> dequant code * 2eb), then each chunk's outliers are written
+ * back over the reconstruction.                                            */
 int orc_decompress(const uint8_t *s, uint64_t bytes, float *out, uint64_t n_expected) {
     orc_header h;
     int rc = orc_parse_header(s, bytes, &h);
@@ -444,32 +452,47 @@ int orc_decompress(const uint8_t *s, uint64_t bytes, float *out, uint64_t n_expe
     if (h.n != n_expected) return ORC_ERR_ARG;
 
     uint32_t words[256], z[256];
-    uint64_t word_off = 0;
-    for (uint64_t b = 0; b < h.nb; ++b) {
-        uint64_t first = b * h.block;
-        uint32_t cnt = (uint32_t)((h.n - first < h.block) ? (h.n - first) : h.block);
-        uint32_t w = s[h.width_off + b];
-        if (w > 32) return ORC_ERR_CORRUPT;
-        uint32_t nw = orc_block_words(w, cnt);
-        if (word_off + nw > h.W) return ORC_ERR_CORRUPT;
-        for (uint32_t k = 0; k < nw; ++k)
-            words[k] = get_u32(s + h.payload_off + 4 * (word_off + k));
-        orc_unpack_block(words, cnt, w, z);
-        int64_t qv = 0; /* undelta: running sum restarting at each block */
-        for (uint32_t j = 0; j < cnt; ++j) {
-            qv += orc_unzigzag(z[j]);
-            int32_t q = (int32_t)(uint32_t)(uint64_t)qv;
-            out[first + j] = dequant(q, h.step);
+    uint64_t blocks_per_chunk = ORC_CHUNK / h.block;
+    uint64_t R = h.W + 2 * h.m, W_seen = 0;
+    for (uint64_t c = 0; c < h.nc; ++c) {
+        uint64_t rec = get_u32(s + h.index_off + 8 * c);
+        uint64_t before = get_u32(s + h.index_off + 8 * c + 4);
+        uint64_t rec_next = (c + 1 < h.nc) ? get_u32(s + h.index_off + 8 * (c + 1)) : R;
+        uint64_t after = (c + 1 < h.nc) ? get_u32(s + h.index_off + 8 * (c + 1) + 4) : h.m;
+        if (rec_next < rec || after < before || rec_next > R || after > h.m) return ORC_ERR_CORRUPT;
+        uint64_t mc = after - before;
+        uint64_t word_off = rec;
+        uint64_t b_end = (c + 1) * blocks_per_chunk < h.nb ? (c + 1) * blocks_per_chunk : h.nb;
+        for (uint64_t b = c * blocks_per_chunk; b < b_end; ++b) {
+            uint64_t first = b * h.block;
+            uint32_t cnt = (uint32_t)((h.n - first < h.block) ? (h.n - first) : h.block);
+            uint32_t w = s[h.width_off + b];
+            if (w > 32) return ORC_ERR_CORRUPT;
+            uint32_t nw = orc_block_words(w, cnt);
+            if (word_off + nw > rec_next) return ORC_ERR_CORRUPT;
+            for (uint32_t k = 0; k < nw; ++k)
+                words[k] = get_u32(s + h.record_off + 4 * (word_off + k));
+            orc_unpack_block(words, cnt, w, z);
+            int64_t qv = 0; /* undelta: running sum restarting at each block */
+            for (uint32_t j = 0; j < cnt; ++j) {
+                qv += orc_unzigzag(z[j]);
+                int32_t q = (int32_t)(uint32_t)(uint64_t)qv;
+                out[first + j] = dequant(q, h.step);
+            }
+            word_off += nw;
         }
-        word_off += nw;
+        if (word_off + 2 * mc != rec_next) return ORC_ERR_CORRUPT;
+        W_seen += word_off - rec;
+        uint64_t e_first = c * ORC_CHUNK;
+        uint64_t e_end = e_first + ORC_CHUNK < h.n ? e_first + ORC_CHUNK : h.n;
+        for (uint64_t k = 0; k < mc; ++k) {
+            uint32_t i = get_u32(s + h.record_off + 4 * (word_off + k));
+            uint32_t bits = get_u32(s + h.record_off + 4 * (word_off + mc + k));
+            if (i < e_first || i >= e_end) return ORC_ERR_CORRUPT;
+            memcpy(&out[i], &bits, 4);
+        }
     }
-    if (word_off != h.W) return ORC_ERR_CORRUPT;
-    for (uint64_t k = 0; k < h.m; ++k) {
-        uint32_t i = get_u32(s + h.idx_off + 4 * k);
-        uint32_t bits = get_u32(s + h.val_off + 4 * k);
-        if (i >= h.n) return ORC_ERR_CORRUPT;
-        memcpy(&out[i], &bits, 4);
-    }
+    if (W_seen != h.W) return ORC_ERR_CORRUPT;
     return 0;
 }
 

@@ -32,10 +32,8 @@ def header(stream) -> dict:
 def sections(h: dict) -> dict:
     w_off = 128
     i_off = w_off + pad16(h["nb"])
-    p_off = i_off + pad16(8 * h["nc"])
-    x_off = p_off + pad16(4 * h["W"])
-    v_off = x_off + pad16(4 * h["m"])
-    return dict(width=w_off, index=i_off, payload=p_off, idx=x_off, val=v_off, total=v_off + 4 * h["m"])
+    r_off = i_off + pad16(8 * h["nc"])
+    return dict(width=w_off, index=i_off, record=r_off, total=r_off + 4 * (h["W"] + 2 * h["m"]))
 
 
 def block_counts(n: int, block: int) -> np.ndarray:
@@ -47,16 +45,34 @@ def block_counts(n: int, block: int) -> np.ndarray:
 
 
 def parts(stream) -> dict:
+    """Split a stream into its sections.  Records are walked chunk by chunk
+    with the widths (payload words of each block) and the chunk index
+    (outliers per chunk); payload words of all chunks are concatenated, and so
+    are the outlier index and value arrays."""
     s = np.asarray(stream, dtype=np.uint8)
     h = header(s)
     off = sections(h)
     widths = s[off["width"]:off["width"] + h["nb"]].astype(np.int64)
-    index = s[off["index"]:off["index"] + 8 * h["nc"]].view(np.uint32).reshape(-1, 2) if h["nc"] else \
-        np.zeros((0, 2), np.uint32)
-    payload = s[off["payload"]:off["payload"] + 4 * h["W"]]
-    idx = s[off["idx"]:off["idx"] + 4 * h["m"]].view(np.uint32)
-    val = s[off["val"]:off["val"] + 4 * h["m"]].view(np.uint32)
-    return dict(h=h, off=off, widths=widths, index=index, payload=payload, idx=idx, val=val, raw=s)
+    index = s[off["index"]:off["index"] + 8 * h["nc"]].view(np.uint32).reshape(-1, 2).astype(np.int64) \
+        if h["nc"] else np.zeros((0, 2), np.int64)
+    rec = s[off["record"]:off["total"]].view(np.uint32)
+    cnt = block_counts(h["n"], h["block"])
+    bwords = -(-(widths * cnt) // 32)
+    bpc = CHUNK // h["block"]
+    payload, idx, val, chunk_m, chunk_words = [], [], [], [], []
+    for c in range(h["nc"]):
+        r0 = int(index[c, 0])
+        m_c = (int(index[c + 1, 1]) if c + 1 < h["nc"] else h["m"]) - int(index[c, 1])
+        pw = int(bwords[c * bpc:(c + 1) * bpc].sum())
+        payload.append(rec[r0:r0 + pw])
+        idx.append(rec[r0 + pw:r0 + pw + m_c])
+        val.append(rec[r0 + pw + m_c:r0 + pw + 2 * m_c])
+        chunk_m.append(m_c)
+        chunk_words.append(pw)
+    cat = lambda a: np.concatenate(a).astype(np.uint32) if a else np.zeros(0, np.uint32)
+    return dict(h=h, off=off, widths=widths, index=index, payload=cat(payload).view(np.uint8),
+                idx=cat(idx), val=cat(val), raw=s, chunk_m=np.array(chunk_m, np.int64),
+                chunk_words=np.array(chunk_words, np.int64), block_words=bwords)
 
 
 def decode_codes_bitmatrix(stream) -> np.ndarray:

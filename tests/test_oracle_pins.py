@@ -32,19 +32,19 @@ def test_worked_example_by_hand(orc):
     [0, 4, 4, 1, 7]; OR = 7 so w = 3; bits (LSB first) 0 | 4<<3 | 4<<6 | 1<<9
     | 7<<12 = 32 + 256 + 512 + 28672 = 29472 = 0x00007320: one word.
     Layout: header 128 B, width byte at 128 padded to 144, one chunk index
-    pair (0, 0) at 144 padded to 160, payload word at 160 padded to 176, no
-    outliers: total 176 bytes."""
+    pair (0, 0) at 144 padded to 160, the chunk record (one payload word, no
+    outliers) at 160: total 164 bytes."""
     x = np.array([0, 2, 4, 3, -1], np.float32)
     s = orc.compress(x, 32, abs=0.5)
-    assert s.size == 176
+    assert s.size == 164
     h = SC.header(s)
     assert (h["magic"], h["version"], h["flags"], h["n"], h["block"], h["chunk"]) == (0x434C4245, 1, 1, 5, 32, 4096)
     assert (h["eb"], h["inv2eb"], h["step"], h["vmin"], h["vmax"]) == (0.5, 1.0, 1.0, 0.0, 0.0)
-    assert (h["nb"], h["nc"], h["W"], h["m"], h["total"], h["bound"]) == (1, 1, 1, 0, 176, 0.5)
+    assert (h["nb"], h["nc"], h["W"], h["m"], h["total"], h["bound"]) == (1, 1, 1, 0, 164, 0.5)
     assert h["reserved"] == bytes(32)
     assert list(s[128:144]) == [3] + [0] * 15
     assert list(s[144:160]) == [0] * 16
-    assert list(s[160:176]) == [0x20, 0x73, 0, 0] + [0] * 12
+    assert list(s[160:164]) == [0x20, 0x73, 0, 0]
     assert orc.decompress(s, 5).tolist() == [0, 2, 4, 3, -1]
 
 
@@ -56,16 +56,18 @@ def test_worked_example_relative_and_outlier(orc):
     even), 1, 0 (non-finite)].  x' = [0, 4, 2, 0]: errors 1, 1, 0.75 <= eb,
     nan is an outlier.  deltas [0, 2, -1, -1] -> zigzag [0, 4, 1, 1], w = 3,
     word = 0 | 4<<3 | 1<<6 | 1<<9 = 32 + 64 + 512 = 608 = 0x260.  One outlier
-    (3, nan bits) -> idx at 176 (padded to 192), val at 192, total 196."""
+    (3, nan bits): the record at 160 holds the payload word, then idx 3 at
+    164, then the nan bits at 168: total 172."""
     x = np.array([-1.0, 3.0, 1.25, np.nan], np.float32)
     s = orc.compress(x, 32, rel=0.25)
     h = SC.header(s)
     assert (h["eb"], h["inv2eb"], h["step"], h["vmin"], h["vmax"]) == (1.0, 0.5, 2.0, -1.0, 3.0)
-    assert (h["W"], h["m"], h["total"]) == (1, 1, 196)
+    assert (h["W"], h["m"], h["total"]) == (1, 1, 172)
     assert s[128] == 3
     assert list(s[160:164]) == [0x60, 0x02, 0, 0]
-    assert s[176:180].view(np.uint32)[0] == 3
-    assert s[192:196].view(np.uint32)[0] == np.float32(np.nan).view(np.uint32)
+    assert list(s[144:160]) == [0] * 16
+    assert s[164:168].view(np.uint32)[0] == 3
+    assert s[168:172].view(np.uint32)[0] == np.float32(np.nan).view(np.uint32)
     y = orc.decompress(s, 4)
     assert y[:3].tolist() == [0.0, 4.0, 2.0] and np.isnan(y[3])
 
@@ -260,18 +262,18 @@ def _check_stream(orc, x, s, block, eb_expected=None):
     assert h["m"] == int(flag.sum())
     assert np.array_equal(P["idx"], np.flatnonzero(flag).astype(np.uint32))
     assert np.array_equal(P["val"], x.view(np.uint32)[flag])
-    # chunk index: word offset and outliers before each chunk
-    starts = np.concatenate([[0], np.cumsum(words)])
+    # chunk index: record word offset and outliers before each chunk
+    per_chunk_m = np.add.reduceat(flag.astype(np.int64), np.arange(0, n, SC.CHUNK)) if n else np.zeros(0, np.int64)
     bpc = SC.CHUNK // block
-    for c in range(h["nc"]):
-        assert P["index"][c, 0] == starts[c * bpc]
-        assert P["index"][c, 1] == int(flag[: c * SC.CHUNK].sum())
+    chunk_words = np.add.reduceat(words, np.arange(0, cnt.size, bpc)) if cnt.size else np.zeros(0, np.int64)
+    rec_sizes = chunk_words + 2 * per_chunk_m
+    assert np.array_equal(P["index"][:, 0], np.concatenate([[0], np.cumsum(rec_sizes)])[:-1])
+    assert np.array_equal(P["index"][:, 1], np.concatenate([[0], np.cumsum(per_chunk_m)])[:-1])
+    assert np.array_equal(P["chunk_m"], per_chunk_m)
     # padding bytes are zero
     raw = P["raw"]
     assert not raw[off["width"] + h["nb"]:off["index"]].any()
-    assert not raw[off["index"] + 8 * h["nc"]:off["payload"]].any()
-    assert not raw[off["payload"] + 4 * h["W"]:off["idx"]].any()
-    assert not raw[off["idx"] + 4 * h["m"]:off["val"]].any()
+    assert not raw[off["index"] + 8 * h["nc"]:off["record"]].any()
     # reconstruction: within eb in fp64 for non-outliers, outliers bit-exact
     y = orc.decompress(s, n)
     keep = ~flag
