@@ -1,0 +1,427 @@
+"""Benchmark: compress + decompress throughput of float32 input on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-cpu-baseline]
+
+One step = one pass of the whole hot path over the workload: value range,
+fused encode (one stream), fused decode.  Default workload: the 512^3 k^-3
+field with 1 % spikes and 1e-6 NaN/+-Inf (relative bound 1e-3, block 64).
+With torchrun (N > 1) every rank compresses its own replica of the workload
+(independent arrays, no collective on the data path: weak scaling); the
+timing is the max over ranks.
+
+Printed JSON line (rank 0):
+  value        GB/s of float32 input per compress + decompress round trip,
+               device-resident input, CUDA events around the library calls;
+               the L2 is flushed (256 MiB write) before every call and the
+               flush is not timed
+  e2e          the same through the HOST execution kind (host buffers,
+               host<->device copies inside the timed region)
+  roofline     the dominant kernel against the measured copy bandwidth
+  cpu_baseline the CPU oracle on a bounded sample of the workload
+--impl reference times the CPU oracle itself (the only reference there is).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "compress & decompress GB/s of fp32 input on 1 B200, % of HBM roofline; ratio"
+DEFAULT_WORKLOAD = "field512cube_spikes"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+CPU_SAMPLE_ELEMS = 1 << 24  # 64 MiB of the workload for the CPU oracle legs
+
+
+# ----------------------------------------------------------------------------------------------
+# rank plumbing
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    return int(os.environ.get("RANK", "0")), ws, int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of a list of floats over all ranks (identity for one rank)."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def sum_over_ranks(values, world: int, device=None):
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t.cpu().tolist()
+
+
+# ----------------------------------------------------------------------------------------------
+# clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [p.strip() for p in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------------------------
+# workload
+
+def workload(name: str):
+    from error_bounded_lossy_encode_b200 import workloads as WL
+
+    x = WL.standard(name)
+    o = WL.options_of(name)
+    block = o.pop("block")
+    mode, bound = next(iter(o.items()))
+    return x, block, mode, bound
+
+
+def options_string(block, mode, bound, timing=False):
+    return f"{mode}={bound!r},block={block}" + (",timing=1" if timing else "")
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha(kernel: str) -> str:
+    csrc = os.path.join(ROOT, "error_bounded_lossy_encode_b200", "csrc")
+    h = hashlib.sha256()
+    for f in (f"{kernel}.cu", "common.cuh", "kernels.h"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload_name}.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("source_sha") != kernel_source_sha(kernel):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------------------------
+# CPU oracle legs
+
+def cpu_oracle_sample(x, block, mode, bound, repeats=1):
+    import oracle
+
+    oracle.build()
+    s = x[:CPU_SAMPLE_ELEMS]
+    t_c = t_d = 0.0
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        stream = oracle.compress(s, block, **{mode: bound})
+        t1 = time.perf_counter()
+        oracle.decompress(stream, s.size)
+        t2 = time.perf_counter()
+        t_c += t1 - t0
+        t_d += t2 - t1
+    gbs = repeats * 4 * s.size / (t_c + t_d) / 1e9
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {s.size} elements ({4 * s.size >> 20} MiB) of the workload, compress+decompress, "
+                      f"single-threaded plain C oracle",
+            "compress_gbs": round(repeats * 4 * s.size / t_c / 1e9, 4),
+            "decompress_gbs": round(repeats * 4 * s.size / t_d / 1e9, 4)}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    x, block, mode, bound = workload(args.workload)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(x, block, mode, bound)
+    t0 = time.perf_counter()
+    base = cpu_oracle_sample(x, block, mode, bound, repeats=args.steps)
+    elapsed = time.perf_counter() - t0
+    line = {"metric": METRIC, "value": base["value"], "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * elapsed / max(1, args.steps), 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": args.workload, "n": int(min(x.size, CPU_SAMPLE_ELEMS)), "block": block,
+                       mode: bound, "sample_of_elements": int(x.size)},
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------------------
+# our arm
+
+def run_ours(args):
+    import torch
+
+    import error_bounded_lossy_encode_b200 as E
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    x_np, block, mode, bound = workload(args.workload)
+    n = x_np.size
+    st, plan = E.eblc_plan_create([n], None, options_string(block, mode, bound, timing=True))
+    if st != E.EBLC_OK:
+        raise RuntimeError("plan_create: " + E.STATUS_NAMES[st])
+    _, lim = E.eblc_plan_get_limits(plan)
+    cap = lim["max_compressed_bytes"]
+
+    x = torch.from_numpy(x_np).to(dev)
+    out = torch.empty(cap, dtype=torch.uint8, device=dev)
+    y = torch.empty(n, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ex = E.cuda_exec(stream.cuda_stream)
+    sc = E.eblc_sidecar_t()
+    launches_per_step = (2 if mode == "rel" else 1) + 1
+
+    def step(timed):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        st, nbytes = E.eblc_compress(plan, ex, x.data_ptr(), out.data_ptr(), cap, sc)
+        e1.record(stream)
+        if st != E.EBLC_OK:
+            raise RuntimeError("compress: " + E.STATUS_NAMES[st])
+        _, kc = E.eblc_plan_kernel_times(plan)
+        kc = [(("compress_call" if k == "call" else k), ms, l) for k, ms, l in kc]
+        flush.fill_(2)
+        e2.record(stream)
+        st = E.eblc_decompress(plan, ex, out.data_ptr(), nbytes, sc, y.data_ptr())
+        e3.record(stream)
+        if st != E.EBLC_OK:
+            raise RuntimeError("decompress: " + E.STATUS_NAMES[st])
+        _, kd = E.eblc_plan_kernel_times(plan)
+        kd = [(("decompress_call" if k == "call" else k), ms, l) for k, ms, l in kd]
+        return e0, e1, e2, e3, nbytes, {k: ms for k, ms, _ in kc + kd}
+
+    for _ in range(max(3, args.warmup)):
+        step(False)
+    torch.cuda.synchronize()
+    if E.eblc_check(plan, ex) != E.EBLC_OK:
+        raise RuntimeError("device reported an error during warm-up")
+
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+    recs = [step(True) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+
+    # device time of the library calls (first launch to last device operation)
+    t_comp = sum(r[5]["compress_call"] for r in recs) / 1e3
+    t_dec = sum(r[5]["decompress_call"] for r in recs) / 1e3
+    # the same bracketed by torch events from Python (includes host return latency)
+    t_comp_api = sum(r[0].elapsed_time(r[1]) for r in recs) / 1e3
+    t_dec_api = sum(r[2].elapsed_time(r[3]) for r in recs) / 1e3
+    nbytes = recs[-1][4]
+    kern = {}
+    for r in recs:
+        for k, ms in r[5].items():
+            if not k.endswith("_call"):
+                kern.setdefault(k, []).append(ms)
+    t_comp, t_dec, t_comp_api, t_dec_api = max_over_ranks([t_comp, t_dec, t_comp_api, t_dec_api], world, dev)
+    total_in_bytes = sum_over_ranks([4.0 * n * args.steps], world, dev)[0]
+    step_s = (t_comp + t_dec) / args.steps
+
+    # e2e: HOST execution kind, pinned host buffers, copies inside the timed region
+    xh = torch.from_numpy(x_np).pin_memory()
+    sh = torch.empty(cap, dtype=torch.uint8).pin_memory()
+    yh = torch.empty(n, dtype=torch.float32).pin_memory()
+    hx = E.host_exec()
+    sc2 = E.eblc_sidecar_t()
+    for _ in range(2):
+        E.eblc_compress(plan, hx, xh.data_ptr(), sh.data_ptr(), cap, sc2)
+    t_e2e = 0.0
+    e2e_steps = max(1, min(args.steps, 5))
+    for _ in range(e2e_steps):
+        t0 = time.perf_counter()
+        st, nb2 = E.eblc_compress(plan, hx, xh.data_ptr(), sh.data_ptr(), cap, sc2)
+        st2 = E.eblc_decompress(plan, hx, sh.data_ptr(), nb2, sc2, yh.data_ptr())
+        t_e2e += time.perf_counter() - t0
+        if st != E.EBLC_OK or st2 != E.EBLC_OK:
+            raise RuntimeError("host-kind call failed")
+    (t_e2e,) = max_over_ranks([t_e2e], world, dev)
+    e2e_bytes = sum_over_ranks([4.0 * n * e2e_steps], world, dev)[0]
+
+    if rank == 0:
+        peak, peak_kind = measured_peak()
+        ratio = 4.0 * n / nbytes
+        comp_gbs = 4.0 * n * args.steps / t_comp / 1e9
+        dec_gbs = 4.0 * n * args.steps / t_dec / 1e9
+        algo = {"range": 4.0 * n, "encode": 4.0 * n + nbytes, "decode": 4.0 * n + nbytes}
+        kstats = {}
+        for k, v in kern.items():
+            avg_ms = float(np.mean(v))
+            ach = algo[k] / (avg_ms / 1e3) / 1e9
+            kstats[k] = {"avg_ms": round(avg_ms, 4), "launches": len(v), "algorithmic_bytes": int(algo[k]),
+                         "achieved_gbs": round(ach, 1), "frac_of_measured_peak": round(ach / peak, 4)}
+        dom = max(kstats, key=lambda k: kstats[k]["avg_ms"])
+        traffic = profiled_traffic(dom, args.workload)
+        line = {
+            "metric": METRIC,
+            "value": round(total_in_bytes / (t_comp + t_dec) / 1e9 * (1 if world == 1 else 1), 2),
+            "unit": "GB/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": max(3, args.warmup),
+            "ms_per_step": round(1e3 * step_s, 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "n": int(n), "block": block, mode: bound,
+                       "l2": "flushed (256 MiB write, untimed) before every compress and decompress call",
+                       "parallelism": f"replicas{world}"},
+            "compress_gbs": round(comp_gbs, 2),
+            "decompress_gbs": round(dec_gbs, 2),
+            "api_ms_per_step": {"compress": round(1e3 * t_comp_api / args.steps, 4),
+                                "decompress": round(1e3 * t_dec_api / args.steps, 4)},
+            "ratio": round(ratio, 4),
+            "stream_bytes": int(nbytes),
+            "hbm_frac_8tbs": {"compress": round((4.0 * n + nbytes) * args.steps / t_comp / 8e12, 4),
+                              "decompress": round((4.0 * n + nbytes) * args.steps / t_dec / 8e12, 4),
+                              "compress_required_bytes": round((8.0 * n + nbytes) * args.steps / t_comp / 8e12, 4)
+                              if mode == "rel" else None},
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": kstats[dom]["achieved_gbs"], "peak": peak,
+                         "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s",
+                         "frac": kstats[dom]["frac_of_measured_peak"], "traffic": traffic},
+            "kernels": kstats,
+            "e2e": {"value": round(e2e_bytes / t_e2e / 1e9, 3), "unit": "GB/s",
+                    "h2d_bytes_per_step": int(4 * n + nb2), "d2h_bytes_per_step": int(nb2 + 4 * n),
+                    "api": "eblc_compress + eblc_decompress, EBLC_EXECUTION_HOST, pinned host buffers"},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+        }
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_oracle_sample(x_np, block, mode, bound)
+        print(json.dumps(line), flush=True)
+    E.eblc_plan_destroy(plan)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

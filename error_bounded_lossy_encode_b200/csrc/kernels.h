@@ -1,0 +1,62 @@
+// kernels.h -- host-side launch interface of the libeblc kernels (internal).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace eblc {
+
+// Value range over the finite elements ("Pipeline specialization
+// internals", Priming: the quantizer's value-range scan before the fused
+// kernel).  Writes range_out[0] = vmin, range_out[1] = vmax (each
+// canonicalised so -0 reads as +0; both 0 when nothing is finite).
+struct RangeArgs {
+    const float *in;   // n floats, 16-byte aligned
+    uint64_t n;
+    float2 *partials;  // one per CTA of the grid
+    uint32_t *counter; // zero on entry; the last CTA resets it
+    float *range_out;  // 2 floats
+};
+int range_grid(int num_sms);
+cudaError_t launch_range(const RangeArgs &a, int grid, cudaStream_t stream);
+
+// Fused encode with single-pass decoupled look-back.  One launch writes the
+// whole stream: header, widths, chunk index and every chunk record.
+struct EncodeArgs {
+    const float *in;          // n floats, 16-byte aligned
+    uint64_t n;
+    uint8_t *out;             // stream buffer, 16-byte aligned
+    uint64_t out_cap;         // bytes available at out
+    uint32_t block;           // 32, 64, 128, 256
+    int abs_mode;
+    double bound;             // relative or absolute bound as requested
+    const float *range;       // vmin, vmax from the range kernel (relative mode)
+    uint64_t *status;         // this call's look-back words [ntiles], zero on entry
+    uint64_t *status_next;    // the other call parity's words, cleared here
+    uint32_t *counter;        // this call's tile counter, zero on entry
+    uint32_t *counter_next;   // cleared here
+    uint32_t *err;            // this call's error word
+    uint32_t *err_next;       // cleared here
+    uint64_t *result;         // [W, m, total, R] written by the last tile
+    uint64_t outlier_cap;
+    int64_t stall_tile;       // test hook (-1: off)
+    uint64_t wait_ns;         // limit of every device-side wait
+};
+cudaError_t launch_encode(const EncodeArgs &a, int num_sms, cudaStream_t stream);
+
+// Fused decode: widths + chunk records -> reconstruction with the chunk's
+// outliers written back.
+struct DecodeArgs {
+    const uint8_t *in;        // stream, 16-byte aligned
+    uint64_t total;           // stream length (validated on the host)
+    uint64_t n;
+    uint32_t block;
+    uint64_t W, m;            // payload words and outliers (from the sidecar)
+    float step;
+    float *out;               // n floats, 16-byte aligned
+    uint32_t *err;            // sticky error word (kErrCorrupt, kErrTimeout)
+    uint64_t wait_ns;
+};
+cudaError_t launch_decode(const DecodeArgs &a, int num_sms, cudaStream_t stream);
+
+}  // namespace eblc

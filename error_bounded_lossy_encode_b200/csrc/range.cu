@@ -1,0 +1,118 @@
+// range.cu -- value range (min, max) over the finite elements.
+//
+// "Pipeline specialization internals", Priming: the quantizer runs a
+// value-range scan and resolves the bound before the fused kernel, because a
+// relative bound eb = rel * (max - min) must be known before any code is
+// produced.  This is the compulsory first read of the input in relative mode.
+//
+// HBM-bound: 4 bytes read per element, no writes.  Persistent grid of
+// 8 CTAs x 256 threads per SM; each thread keeps 4 float4 loads in flight.
+// The array is walked from its end to its start so the lowest addresses are
+// the last read and are still in L2 when the encoder starts at tile 0.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace eblc {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ void fold(float v, float &lo, float &hi) {
+    const bool finite = fabsf(v) < __int_as_float(0x7f800000);  // false for NaN and +-Inf
+    lo = fminf(lo, finite ? v : __int_as_float(0x7f800000));
+    hi = fmaxf(hi, finite ? v : __int_as_float(0xff800000));
+}
+
+__global__ void __launch_bounds__(kThreads) range_kernel(RangeArgs a) {
+    float lo = __int_as_float(0x7f800000), hi = __int_as_float(0xff800000);
+    const float4 *in4 = reinterpret_cast<const float4 *>(a.in);
+    const uint64_t n4 = a.n / 4;
+    const uint64_t stride = (uint64_t)gridDim.x * kThreads;
+    const uint64_t tid = (uint64_t)blockIdx.x * kThreads + threadIdx.x;
+
+    for (uint64_t base = 0; base < n4; base += stride * kUnroll) {
+        float4 v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint64_t i = base + u * stride + tid;
+            v[u] = (i < n4) ? __ldg(in4 + (n4 - 1 - i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const uint64_t i = base + u * stride + tid;
+            if (i < n4) {
+                fold(v[u].x, lo, hi);
+                fold(v[u].y, lo, hi);
+                fold(v[u].z, lo, hi);
+                fold(v[u].w, lo, hi);
+            }
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x < (a.n & 3)) fold(a.in[n4 * 4 + threadIdx.x], lo, hi);
+
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    __shared__ float2 warp_part[kThreads / 32];
+    __shared__ bool is_last;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (lane == 0) warp_part[warp] = make_float2(lo, hi);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kThreads / 32; ++w) {
+            lo = fminf(lo, warp_part[w].x);
+            hi = fmaxf(hi, warp_part[w].y);
+        }
+        a.partials[blockIdx.x] = make_float2(lo, hi);
+        __threadfence();
+        const uint32_t done = atomicAdd(a.counter, 1u);
+        is_last = (done == gridDim.x - 1);
+    }
+    __syncthreads();
+    if (!is_last) return;
+
+    // Last CTA: fold the per-CTA partials (in CTA order) and publish.
+    __threadfence();
+    lo = __int_as_float(0x7f800000);
+    hi = __int_as_float(0xff800000);
+    for (uint32_t i = threadIdx.x; i < gridDim.x; i += kThreads) {
+        const float2 p = __ldcg(a.partials + i);
+        lo = fminf(lo, p.x);
+        hi = fmaxf(hi, p.y);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+    }
+    __syncthreads();
+    if (lane == 0) warp_part[warp] = make_float2(lo, hi);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < kThreads / 32; ++w) {
+            lo = fminf(lo, warp_part[w].x);
+            hi = fmaxf(hi, warp_part[w].y);
+        }
+        if (!(lo <= hi)) {  // no finite element
+            lo = 0.0f;
+            hi = 0.0f;
+        }
+        a.range_out[0] = __fadd_rn(lo, 0.0f);  // canonical +0 for a zero end
+        a.range_out[1] = __fadd_rn(hi, 0.0f);
+        *a.counter = 0;
+    }
+}
+
+}  // namespace
+
+int range_grid(int num_sms) { return num_sms * 8; }
+
+cudaError_t launch_range(const RangeArgs &a, int grid, cudaStream_t stream) {
+    range_kernel<<<grid, kThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace eblc

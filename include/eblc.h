@@ -1,0 +1,223 @@
+/*
+ * eblc.h -- C ABI of libeblc, a B200 (sm_100a) error-bounded lossy
+ * compressor for float32 arrays.
+ *
+ * The hot path is one fused block-local pipeline: linear quantizer ->
+ * 1-D Lorenzo predictor reset at each block -> zigzag -> adaptive
+ * fixed-length bitpack, with an outlier side list, and a cross-block scan
+ * that places every block at its final offset in one stream; plus its exact
+ * inverse.  Every element of the reconstruction x' satisfies
+ * |x - x'| <= eb (tested in IEEE double), non-finite elements and elements
+ * that would break the bound are stored losslessly in the outlier list.
+ *
+ * Sources (page title, section):
+ *   "DevitoComp provider interface" -- "Configuring the error tolerance"
+ *     (a non-negative relative error fixed at plan creation, passed as a
+ *     decimal string or NULL for the provider default), "Provider layout"
+ *     (plan_create with an options string; dims and strides in
+ *     slowest-to-fastest order, strides in elements; HOST / CUDA / HIP
+ *     execution descriptor with an optional native stream; per-snapshot
+ *     host sidecar ready on return; device work may stay queued; providers
+ *     report payload alignment through a limits struct and may return
+ *     UNSUPPORTED), "Dummy provider" (contiguous float32 tensors; a maximum
+ *     compressed size).
+ *   FZGPUModules "Pipeline specialization internals" -- "Roles and
+ *     strategies", "Forward declaration", "Inverse declaration", "Priming:
+ *     the fused runner bypasses execute()" (default bound 1e-4; the inverse
+ *     must read the resolved bound), "The device policy contract".
+ *   "nvrtc_chunk_fusion.h File Reference" -- launchNvrtcChunkFusedEncode and
+ *     launchGenericChunkFusion (outlier side output: uint32 indices + values;
+ *     the cross-chunk scan/pack tail returns the archive byte length after a
+ *     stream synchronisation).
+ *
+ * Threading and streams: a plan may be used by one host thread and one
+ * stream at a time (it owns the scratch memory of its calls).  All device
+ * pointers must belong to the device that was current at eblc_plan_create.
+ *
+ * Errors: every call returns an eblc_status_t; no C++ exception crosses this
+ * ABI and nothing aborts the process.  Device-side faults that the kernels
+ * detect (corrupt stream, capacity, a bounded wait that ran out) are
+ * reported through a device error word, read by eblc_compress (which
+ * synchronises) or by eblc_check.
+ */
+#ifndef EBLC_H
+#define EBLC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(_WIN32)
+#define EBLC_API
+#else
+#define EBLC_API __attribute__((visibility("default")))
+#endif
+
+#define EBLC_ABI_VERSION 1u
+
+typedef enum {
+    EBLC_OK = 0,
+    EBLC_UNSUPPORTED = 1,  /* execution kind, layout or option not supported      */
+    EBLC_INVALID_ARG = 2,  /* bad pointer, size, alignment or option value          */
+    EBLC_CAPACITY = 3,     /* output buffer or outlier capacity too small           */
+    EBLC_CORRUPT = 4,      /* stream or sidecar malformed (host or device detected) */
+    EBLC_CUDA_ERROR = 5,   /* a CUDA runtime call failed                            */
+    EBLC_TIMEOUT = 6,      /* a bounded device-side wait ran out                    */
+    EBLC_NOMEM = 7         /* host or device allocation failed                      */
+} eblc_status_t;
+
+typedef enum {
+    /* Host pointers.  The call is synchronous.  The work still runs on the
+     * GPU: the plan copies the input to device staging buffers, runs the
+     * same kernels, and copies the result back (no CPU code path).
+     * num_threads and stream are ignored.  Pinned host memory is fastest.  */
+    EBLC_EXECUTION_HOST = 0,
+    /* Device pointers on the plan's device, work queued on `stream`
+     * (a cudaStream_t; NULL = the legacy default stream).                   */
+    EBLC_EXECUTION_CUDA = 1,
+    /* Not supported: returns EBLC_UNSUPPORTED.                              */
+    EBLC_EXECUTION_HIP = 2
+} eblc_execution_kind_t;
+
+typedef struct {
+    int32_t kind;        /* eblc_execution_kind_t                     */
+    int32_t num_threads; /* ignored                                   */
+    void *stream;        /* cudaStream_t for EBLC_EXECUTION_CUDA      */
+} eblc_execution_t;
+
+typedef struct eblc_plan_s *eblc_plan_t;
+
+typedef struct {
+    uint64_t n;                    /* elements per snapshot (product of dims)             */
+    uint32_t block;                /* block size B (elements), one of 32, 64, 128, 256    */
+    uint32_t chunk;                /* elements per chunk record (4096)                    */
+    uint64_t max_compressed_bytes; /* worst-case stream size for this plan                */
+    uint64_t payload_alignment;    /* required alignment of stream and float buffers (16) */
+    uint64_t sidecar_bytes;        /* size of the host sidecar (64)                       */
+    uint64_t sidecar_alignment;    /* alignment of the host sidecar (8)                   */
+    uint64_t outlier_capacity;     /* most outliers a stream may hold (default n)         */
+    double bound;                  /* error bound requested (relative or absolute)        */
+    int32_t abs_mode;              /* 1 if `bound` is absolute, 0 if relative             */
+    int32_t reserved;
+} eblc_limits_t;
+
+/* Host sidecar written by eblc_compress (64 bytes, 8-byte aligned, little
+ * endian).  It repeats the stream header fields that a decompressing caller
+ * needs to validate sizes without reading device memory.                    */
+typedef struct {
+    uint32_t magic;         /* 0x434C4245 ("EBLC")                   */
+    uint16_t version;       /* stream version (1)                    */
+    uint16_t flags;         /* bit0: absolute bound                  */
+    uint32_t block;         /* B                                     */
+    uint32_t chunk;         /* 4096                                  */
+    uint64_t n;             /* elements                              */
+    uint64_t total_bytes;   /* stream length                         */
+    uint64_t payload_words; /* W                                     */
+    uint64_t n_outliers;    /* m                                     */
+    double eb;              /* resolved absolute bound               */
+    float step;             /* dequantisation step (float)(2 eb)     */
+    float inv2eb;           /* quantisation factor (float)(1/(2 eb)) */
+} eblc_sidecar_t;
+
+/* Device timing of the last call, recorded when the plan was created with
+ * the option "timing=1": CUDA events on the call's stream around each kernel
+ * launch, plus one entry "call" from the first launch to the end of the
+ * call's last device operation (for compress: the result readback).        */
+typedef struct {
+    char name[24];      /* "range", "encode", "decode", "call"          */
+    float ms;           /* elapsed device time                          */
+    uint32_t launches;  /* 1 for a kernel; kernels in the call for "call" */
+} eblc_kernel_time_t;
+
+/* Version of this ABI (EBLC_ABI_VERSION).                                   */
+EBLC_API uint32_t eblc_abi_version(void);
+
+/* Static description of a status code.                                      */
+EBLC_API const char *eblc_status_string(eblc_status_t status);
+
+/*
+ * Create a plan for float32 snapshots of shape dims[0..rank) (slowest to
+ * fastest).  strides (in elements, slowest to fastest) may be NULL for
+ * C-contiguous data; any non-contiguous stride gives EBLC_UNSUPPORTED.  The
+ * data are coded as one flat sequence in C order.  Requires 1 <= rank <= 8,
+ * dims >= 0 and n = prod(dims) <= 2^30.
+ *
+ * options: NULL -> relative bound 1e-4, block 128.  A bare decimal ("1e-3")
+ * is a relative bound.  Otherwise comma-separated key=value:
+ *   rel=<x>          relative bound, eb = x * (max - min) over the finite
+ *                    elements of each snapshot (x finite, >= 0)
+ *   abs=<x>          absolute bound eb = x (finite, >= 0)
+ *   block=<B>        32 | 64 | 128 | 256 (default 128)
+ *   outlier_cap=<k>  most outliers per stream (default n); more gives
+ *                    EBLC_CAPACITY
+ *   timing=1         record per-kernel device times (eblc_plan_kernel_times)
+ *   wait_ms=<t>      limit of device-side waits in milliseconds (default 2000)
+ *   stall_tile=<t>   test hook: tile t of the next compress never publishes
+ *                    its scan value, so later tiles' waits run out and the
+ *                    call returns EBLC_TIMEOUT (default off)
+ * The plan allocates its device scratch here (cudaMalloc on the current
+ * device).  *out is NULL on failure.
+ */
+EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_t *dims,
+                                        const int64_t *strides, const char *options);
+
+/* Sizes and alignment rules of a plan.                                      */
+EBLC_API eblc_status_t eblc_plan_get_limits(eblc_plan_t plan, eblc_limits_t *out);
+
+/*
+ * Compress one snapshot.
+ *   d_in          n float32 values (device pointer for CUDA kind, host pointer
+ *                 for HOST kind), 16-byte aligned; caller owned, not modified.
+ *   d_out         output buffer of out_capacity bytes, 16-byte aligned
+ *                 (device or host pointer by kind); caller owned.
+ *   out_capacity  bytes available at d_out.  If the stream does not fit the
+ *                 call returns EBLC_CAPACITY and nothing beyond out_capacity
+ *                 is written; max_compressed_bytes always fits.
+ *   compressed_bytes  receives the stream length.
+ *   h_sidecar     host buffer of sidecar_bytes (8-byte aligned) receiving an
+ *                 eblc_sidecar_t; may be NULL.
+ * The call synchronises the stream once at the end (the length and the
+ * sidecar must be ready on return).  Stream layout: see the stream format
+ * notes shipped with this library (header, widths, chunk index, one record
+ * per 4096-element chunk holding its payload words then its outliers).
+ */
+EBLC_API eblc_status_t eblc_compress(eblc_plan_t plan, const eblc_execution_t *exec, const float *d_in,
+                                     void *d_out, size_t out_capacity, size_t *compressed_bytes,
+                                     void *h_sidecar);
+
+/*
+ * Decompress one snapshot.
+ *   d_in              the stream (compressed_bytes long, 16-byte aligned).
+ *   h_sidecar         the sidecar eblc_compress returned with this stream
+ *                     (may be NULL; then the stream header is copied to the
+ *                     host, which synchronises the stream).
+ *   d_out             n float32 values, 16-byte aligned, caller owned.
+ * With the CUDA kind and a sidecar the work stays queued on the stream (no
+ * synchronisation); device-detected corruption is reported by eblc_check.
+ * The stream must have been produced with the same n and block; the bound
+ * is read from the stream, never from the plan.
+ */
+EBLC_API eblc_status_t eblc_decompress(eblc_plan_t plan, const eblc_execution_t *exec, const void *d_in,
+                                       size_t compressed_bytes, const void *h_sidecar, float *d_out);
+
+/* Synchronise exec->stream and return (then clear) the status recorded by
+ * the device during this plan's calls since the last check.                */
+EBLC_API eblc_status_t eblc_check(eblc_plan_t plan, const eblc_execution_t *exec);
+
+/* Device times of the last compress / decompress (option timing=1): one
+ * entry per kernel, then the whole call.  Synchronises on the recorded
+ * events.  Writes at most cap entries and sets *count to the number
+ * written; EBLC_UNSUPPORTED if the plan records no timing.                 */
+EBLC_API eblc_status_t eblc_plan_kernel_times(eblc_plan_t plan, eblc_kernel_time_t *out, int cap, int *count);
+
+/* Release the plan and its device memory.  NULL is allowed.                */
+EBLC_API void eblc_plan_destroy(eblc_plan_t plan);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EBLC_H */

@@ -1,0 +1,89 @@
+"""CPU-side checks of the C-ABI library: it builds for sm_100a, loads, and
+exports every entry point include/eblc.h declares; argument and option
+validation that happens before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def E():
+    from error_bounded_lossy_encode_b200 import build
+
+    build.build()
+    import error_bounded_lossy_encode_b200 as E
+
+    return E
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "eblc.h")).read()
+    return sorted(set(re.findall(r"EBLC_API[^;(]*?\b(eblc_\w+)\s*\(", src)))
+
+
+def test_header_declares_entry_points():
+    names = _declared()
+    assert {"eblc_abi_version", "eblc_status_string", "eblc_plan_create", "eblc_plan_get_limits", "eblc_compress",
+            "eblc_decompress", "eblc_check", "eblc_plan_kernel_times", "eblc_plan_destroy"} <= set(names)
+
+
+def test_library_exports_every_declared_symbol(E):
+    L = ctypes.CDLL(E.LIB_PATH)
+    for name in _declared():
+        assert hasattr(L, name), name
+
+
+def test_only_api_symbols_exported(E):
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--defined-only", E.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert {s for s in exported if s.startswith("eblc_")} == set(_declared())
+
+
+def test_version_and_status_strings(E):
+    assert E.eblc_abi_version() == 1
+    assert E.eblc_status_string(E.EBLC_OK) == "ok"
+    assert E.eblc_status_string(E.EBLC_CORRUPT) == "corrupt stream"
+    assert E.eblc_status_string(99) == "unknown status"
+
+
+def test_struct_sizes(E):
+    assert ctypes.sizeof(E.eblc_sidecar_t) == 64
+    assert ctypes.sizeof(E.eblc_limits_t) == 72  # matches the static_assert in plan.cu
+
+
+@pytest.mark.parametrize("opts,status", [
+    ("rel=-1", 2), ("abs=nan", 2), ("rel=1e-3,abs=1e-3", 2), ("block=48", 1), ("bogus=1", 1), ("rel", 2),
+    ("block=x", 2), ("outlier_cap=-3", 2), ("wait_ms=0", 2)])
+def test_option_errors_need_no_gpu(E, opts, status):
+    st, plan = E.eblc_plan_create([100], None, opts)
+    assert st == status and plan is None
+
+
+def test_shape_errors_need_no_gpu(E):
+    assert E.eblc_plan_create([], None, None)[0] == E.EBLC_INVALID_ARG
+    assert E.eblc_plan_create([-1], None, None)[0] == E.EBLC_INVALID_ARG
+    assert E.eblc_plan_create([1 << 20, 1 << 11], None, None)[0] == E.EBLC_UNSUPPORTED
+    assert E.eblc_plan_create([4, 5], [1, 4], None)[0] == E.EBLC_UNSUPPORTED
+
+
+def test_null_arguments(E):
+    assert E.lib().eblc_plan_create(None, 1, None, None, None) == E.EBLC_INVALID_ARG
+    assert E.lib().eblc_plan_get_limits(None, None) == E.EBLC_INVALID_ARG
+    assert E.lib().eblc_compress(None, None, None, None, 0, None, None) == E.EBLC_INVALID_ARG
+    assert E.lib().eblc_decompress(None, None, None, 0, None, None) == E.EBLC_INVALID_ARG
+    E.eblc_plan_destroy(None)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    import error_bounded_lossy_encode_b200 as E
+
+    monkeypatch.setattr(E, "_lib", None)
+    monkeypatch.setattr(E, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        E.lib()
