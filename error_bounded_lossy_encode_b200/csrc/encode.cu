@@ -297,16 +297,13 @@ __device__ __forceinline__ bool finish_tile(EncSmem &sm, const EncodeArgs &a, co
         }
     }
 
-    if (cw == 0) {  // width bytes of the tile (zeros past the last block up to the 16-byte pad)
-        constexpr uint32_t K = kChunk / kB;
-        const uint64_t b0 = (uint64_t)tile * K;
-        const uint64_t bend = min(b0 + K, pad16(L.nb));
-        const uint32_t nwords = (uint32_t)((bend - b0) / 4);
-        const uint32_t *ws = reinterpret_cast<const uint32_t *>(sm.width[q]);
-        uint32_t *wd = reinterpret_cast<uint32_t *>(a.out + L.width_off + b0);
-        for (uint32_t j = ln; j < nwords; j += 32) {
-            if (L.width_off + b0 + 4 * j + 4 <= a.out_cap)
-                wd[j] = ws[j];
+    {  // this warp's width bytes (zeros past the last block up to the 16-byte pad)
+        constexpr uint32_t kBPW = kChunk / kB / kNW;  // blocks per warp per tile
+        const uint64_t b = (uint64_t)tile * (kChunk / kB) + cw * kBPW + ln;
+        const uint64_t off = L.width_off + b;
+        if (ln < (int)kBPW && b < pad16(L.nb)) {
+            if (off < a.out_cap)
+                a.out[off] = sm.width[q][cw * kBPW + ln];
             else
                 over = true;
         }

@@ -169,3 +169,16 @@ def test_cross_decode_oracle_stream(torch_cuda, orc):
             st, chk, y = g.decompress_np(s, None)
             assert st == 0 and chk == 0
             assert bits_equal(y, orc.decompress(s, x.size))
+
+
+@pytest.mark.parametrize("block", BLOCKS)
+def test_parity_many_tiles_per_cta(torch_cuda, orc, block):
+    """Enough 4096-element chunks (about 5 per CTA) that every CTA cycles its
+    shared-memory rings and barrier phases several times, in both kernels."""
+    rng = np.random.default_rng(block)
+    n = 1500 * 4096 + 123
+    x = np.cumsum(rng.standard_normal(n) * 0.02).astype(np.float32)
+    x[rng.random(n) < 1e-4] = np.nan
+    x[rng.random(n) < 1e-3] *= 1e3
+    _run_parity(orc, x, block, rel=1e-3)
+    _run_parity(orc, x, block, abs=1e-4)
