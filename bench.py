@@ -141,10 +141,12 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------------
 # workload
 
-def workload(name: str):
+def workload(name: str, elements: int | None = None):
     from error_bounded_lossy_encode_b200 import workloads as WL
 
     x = WL.standard(name)
+    if elements:
+        x = np.ascontiguousarray(x[:elements])
     o = WL.options_of(name)
     block = o.pop("block")
     mode, bound = next(iter(o.items()))
@@ -216,7 +218,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    x, block, mode, bound = workload(args.workload)
+    x, block, mode, bound = workload(args.workload, args.elements)
     for _ in range(args.warmup):
         cpu_oracle_sample(x, block, mode, bound)
     t0 = time.perf_counter()
@@ -254,7 +256,7 @@ def run_ours(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    x_np, block, mode, bound = workload(args.workload)
+    x_np, block, mode, bound = workload(args.workload, args.elements)
     n = x_np.size
     st, plan = E.eblc_plan_create([n], None, options_string(block, mode, bound, timing=True))
     if st != E.EBLC_OK:
@@ -329,6 +331,24 @@ def run_ours(args):
     step_s = (t_comp + t_dec) / args.steps
 
     # e2e: HOST execution kind, pinned host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(E, plan, x_np, cap, args, world, dev)
+    if rank == 0:
+        report(args, world, n, nbytes, t_comp, t_dec, t_comp_api, t_dec_api, total_in_bytes, step_s, kern, e2e,
+               launches_per_step, clk, x_np, block, mode, bound)
+    E.eblc_plan_destroy(plan)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(E, plan, x_np, cap, args, world, dev):
+    import torch
+
+    n = x_np.size
     xh = torch.from_numpy(x_np).pin_memory()
     sh = torch.empty(cap, dtype=torch.uint8).pin_memory()
     yh = torch.empty(n, dtype=torch.float32).pin_memory()
@@ -347,66 +367,64 @@ def run_ours(args):
             raise RuntimeError("host-kind call failed")
     (t_e2e,) = max_over_ranks([t_e2e], world, dev)
     e2e_bytes = sum_over_ranks([4.0 * n * e2e_steps], world, dev)[0]
+    return {"value": round(e2e_bytes / t_e2e / 1e9, 3), "unit": "GB/s",
+            "h2d_bytes_per_step": int(4 * n + nb2), "d2h_bytes_per_step": int(nb2 + 4 * n),
+            "api": "eblc_compress + eblc_decompress, EBLC_EXECUTION_HOST, pinned host buffers"}
 
-    if rank == 0:
-        peak, peak_kind = measured_peak()
-        ratio = 4.0 * n / nbytes
-        comp_gbs = 4.0 * n * args.steps / t_comp / 1e9
-        dec_gbs = 4.0 * n * args.steps / t_dec / 1e9
-        algo = {"range": 4.0 * n, "encode": 4.0 * n + nbytes, "decode": 4.0 * n + nbytes}
-        kstats = {}
-        for k, v in kern.items():
-            avg_ms = float(np.mean(v))
-            ach = algo[k] / (avg_ms / 1e3) / 1e9
-            kstats[k] = {"avg_ms": round(avg_ms, 4), "launches": len(v), "algorithmic_bytes": int(algo[k]),
-                         "achieved_gbs": round(ach, 1), "frac_of_measured_peak": round(ach / peak, 4)}
-        dom = max(kstats, key=lambda k: kstats[k]["avg_ms"])
-        traffic = profiled_traffic(dom, args.workload)
-        line = {
-            "metric": METRIC,
-            "value": round(total_in_bytes / (t_comp + t_dec) / 1e9 * (1 if world == 1 else 1), 2),
-            "unit": "GB/s",
-            "n_gpus": world,
-            "steps": args.steps,
-            "warmup": max(3, args.warmup),
-            "ms_per_step": round(1e3 * step_s, 4),
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "f32",
-            "data": "synthetic",
-            "config": {"workload": args.workload, "n": int(n), "block": block, mode: bound,
-                       "l2": "flushed (256 MiB write, untimed) before every compress and decompress call",
-                       "parallelism": f"replicas{world}"},
-            "compress_gbs": round(comp_gbs, 2),
-            "decompress_gbs": round(dec_gbs, 2),
-            "api_ms_per_step": {"compress": round(1e3 * t_comp_api / args.steps, 4),
-                                "decompress": round(1e3 * t_dec_api / args.steps, 4)},
-            "ratio": round(ratio, 4),
-            "stream_bytes": int(nbytes),
-            "hbm_frac_8tbs": {"compress": round((4.0 * n + nbytes) * args.steps / t_comp / 8e12, 4),
-                              "decompress": round((4.0 * n + nbytes) * args.steps / t_dec / 8e12, 4),
-                              "compress_required_bytes": round((8.0 * n + nbytes) * args.steps / t_comp / 8e12, 4)
-                              if mode == "rel" else None},
-            "roofline": {"bound": "hbm", "kernel": dom, "achieved": kstats[dom]["achieved_gbs"], "peak": peak,
-                         "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s",
-                         "frac": kstats[dom]["frac_of_measured_peak"], "traffic": traffic},
-            "kernels": kstats,
-            "e2e": {"value": round(e2e_bytes / t_e2e / 1e9, 3), "unit": "GB/s",
-                    "h2d_bytes_per_step": int(4 * n + nb2), "d2h_bytes_per_step": int(nb2 + 4 * n),
-                    "api": "eblc_compress + eblc_decompress, EBLC_EXECUTION_HOST, pinned host buffers"},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clk,
-        }
-        if not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_oracle_sample(x_np, block, mode, bound)
-        print(json.dumps(line), flush=True)
-    E.eblc_plan_destroy(plan)
-    if world > 1:
-        import torch.distributed as dist
 
-        dist.destroy_process_group()
-    return 0
+def report(args, world, n, nbytes, t_comp, t_dec, t_comp_api, t_dec_api, total_in_bytes, step_s, kern, e2e,
+           launches_per_step, clk, x_np, block, mode, bound):
+    peak, peak_kind = measured_peak()
+    ratio = 4.0 * n / nbytes
+    comp_gbs = 4.0 * n * args.steps / t_comp / 1e9
+    dec_gbs = 4.0 * n * args.steps / t_dec / 1e9
+    algo = {"range": 4.0 * n, "encode": 4.0 * n + nbytes, "decode": 4.0 * n + nbytes}
+    kstats = {}
+    for k, v in kern.items():
+        avg_ms = float(np.mean(v))
+        ach = algo[k] / (avg_ms / 1e3) / 1e9
+        kstats[k] = {"avg_ms": round(avg_ms, 4), "launches": len(v), "algorithmic_bytes": int(algo[k]),
+                     "achieved_gbs": round(ach, 1), "frac_of_measured_peak": round(ach / peak, 4)}
+    dom = max(kstats, key=lambda k: kstats[k]["avg_ms"])
+    traffic = profiled_traffic(dom, args.workload)
+    line = {
+        "metric": METRIC,
+        "value": round(total_in_bytes / (t_comp + t_dec) / 1e9, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(3, args.warmup),
+        "ms_per_step": round(1e3 * step_s, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": args.workload if not args.elements else f"{args.workload}[:{n}]",
+                   "n": int(n), "block": block, mode: bound,
+                   "l2": "flushed (256 MiB write, untimed) before every compress and decompress call",
+                   "parallelism": f"replicas{world}"},
+        "compress_gbs": round(comp_gbs, 2),
+        "decompress_gbs": round(dec_gbs, 2),
+        "api_ms_per_step": {"compress": round(1e3 * t_comp_api / args.steps, 4),
+                            "decompress": round(1e3 * t_dec_api / args.steps, 4)},
+        "ratio": round(ratio, 4),
+        "stream_bytes": int(nbytes),
+        "hbm_frac_8tbs": {"compress": round((4.0 * n + nbytes) * args.steps / t_comp / 8e12, 4),
+                          "decompress": round((4.0 * n + nbytes) * args.steps / t_dec / 8e12, 4),
+                          "compress_required_bytes": round((8.0 * n + nbytes) * args.steps / t_comp / 8e12, 4)
+                          if mode == "rel" else None},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": kstats[dom]["achieved_gbs"], "peak": peak,
+                     "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s",
+                     "frac": kstats[dom]["frac_of_measured_peak"], "traffic": traffic},
+        "kernels": kstats,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(x_np, block, mode, bound)
+    print(json.dumps(line), flush=True)
 
 
 def main(argv=None):
@@ -417,6 +435,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--elements", type=int, default=None, help="use only the first N elements of the workload")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)

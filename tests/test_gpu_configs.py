@@ -37,10 +37,13 @@ def _full_check(orc, x, block, **mode):
     P = SC.parts(want)
     outl = np.zeros(x.size, bool)
     outl[P["idx"]] = True
-    keep = ~outl
-    err = np.abs(x[keep].astype(np.float64) - y[keep].astype(np.float64))
-    assert err.max(initial=0.0) <= h["eb"]
-    assert np.array_equal(y.view(np.uint32)[outl], x.view(np.uint32)[outl])
+    step = 1 << 24
+    for s0 in range(0, x.size, step):  # chunked: fp64 temporaries stay small
+        sl = slice(s0, s0 + step)
+        keep = ~outl[sl]
+        err = np.abs(x[sl][keep].astype(np.float64) - y[sl][keep].astype(np.float64))
+        assert err.max(initial=0.0) <= h["eb"]
+        assert np.array_equal(y[sl].view(np.uint32)[~keep], x[sl].view(np.uint32)[~keep])
     return h
 
 
