@@ -95,6 +95,9 @@ def lib() -> ctypes.CDLL:
     L.eblc_plan_kernel_times.restype = i32
     L.eblc_plan_destroy.argtypes = [P]
     L.eblc_plan_destroy.restype = None
+    L.eblc_compress_noalloc.argtypes = [P, u64, ctypes.c_uint32, i32, ctypes.c_double, P, ctypes.c_size_t, P,
+                                        ctypes.POINTER(ctypes.c_size_t), P]
+    L.eblc_compress_noalloc.restype = i32
     _lib = L
     return L
 
@@ -159,6 +162,20 @@ def eblc_plan_kernel_times(plan, cap: int = 8):
 def eblc_plan_destroy(plan) -> None:
     if plan is not None:
         lib().eblc_plan_destroy(plan)
+
+
+EBLC_NOALLOC_MAX_N = 1 << 26
+
+
+def eblc_compress_noalloc(d_in: int, n: int, block: int, abs_mode: bool, bound: float, d_out: int,
+                          out_capacity: int, stream: int = 0, sidecar=None):
+    """Plan-free compress that allocates no device memory (see include/eblc.h).
+    Returns (status, compressed_bytes)."""
+    nbytes = ctypes.c_size_t(0)
+    st = lib().eblc_compress_noalloc(ctypes.c_void_p(d_in or None), n, block, int(bool(abs_mode)), float(bound),
+                                     ctypes.c_void_p(d_out or None), out_capacity, ctypes.c_void_p(stream or None),
+                                     ctypes.byref(nbytes), None if sidecar is None else ctypes.byref(sidecar))
+    return st, int(nbytes.value)
 
 
 def sidecar_dict(sc: eblc_sidecar_t) -> dict:

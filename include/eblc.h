@@ -216,6 +216,40 @@ EBLC_API eblc_status_t eblc_plan_kernel_times(eblc_plan_t plan, eblc_kernel_time
 /* Release the plan and its device memory.  NULL is allowed.                */
 EBLC_API void eblc_plan_destroy(eblc_plan_t plan);
 
+/* Largest n accepted by eblc_compress_noalloc: 2^26 elements (256 MiB of
+ * float32).  Its scratch is one fixed device array of about 280 KB.        */
+#define EBLC_NOALLOC_MAX_N (1ull << 26)
+
+/*
+ * Compress one array without allocating any device memory.  The paper has
+ * no counterpart to this entry point.  It is for callers that cannot call
+ * cudaMalloc: code running under an allocator that owns all device memory,
+ * code inside a region where an allocation is forbidden or would
+ * synchronise the device, and callers that must not grow the device
+ * footprint behind their back.  No plan is needed; the result is
+ * byte-identical to eblc_plan_create(n, "rel=|abs=<bound>,block=<block>")
+ * followed by eblc_compress.
+ *   d_in, n        n float32 values in device memory, 16-byte aligned;
+ *                  n <= EBLC_NOALLOC_MAX_N, else EBLC_UNSUPPORTED (a message
+ *                  goes to stderr)
+ *   block          32, 64, 128 or 256
+ *   abs_mode, bound  absolute (abs_mode != 0) or relative bound, finite >= 0
+ *   d_out, out_capacity  caller-owned device output, 16-byte aligned
+ *   stream         cudaStream_t (NULL: the legacy default stream)
+ *   compressed_bytes, h_sidecar  as for eblc_compress (h_sidecar may be NULL)
+ * The scratch of the range and encode kernels is a file-scope __device__
+ * array that every GPU that loads this library holds until the process
+ * exits.  The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call on a device shares the array and each call clears what must
+ * start at zero, so calls that overlap on the GPU (other streams, other
+ * host threads) race: serialise them.  Like eblc_compress, the call
+ * synchronises `stream` once at the end.
+ */
+EBLC_API eblc_status_t eblc_compress_noalloc(const float *d_in, uint64_t n, uint32_t block, int abs_mode,
+                                             double bound, void *d_out, size_t out_capacity, void *stream,
+                                             size_t *compressed_bytes, void *h_sidecar);
+
 #ifdef __cplusplus
 }
 #endif
