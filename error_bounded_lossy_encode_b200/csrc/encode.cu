@@ -13,23 +13,29 @@
 //   (launchGenericChunkFusion: scan/pack tail) -- here a single-pass
 //   decoupled look-back instead of a separate scan and gather.
 //
-// CTA organisation (320 threads, 2 CTAs per SM):
-//   warps 0..7  compute: each owns a contiguous 512-element slice of the
-//               4096-element tile, held as warp-tiles of 32*V elements
-//               (V consecutive elements per lane, V = 4, or 8 for B = 256);
-//               a block of B elements spans LPB = B/V lanes.
-//   warp 8      look-back: sums the warp totals of a tile, publishes the
-//               tile aggregate, resolves its exclusive prefix from the
-//               predecessors' status words, writes the chunk index entry
-//               (and the header for the last tile).
-//   warp 9      producer: claims tiles in order from a global counter and
-//               streams them into a 4-stage shared-memory ring with bulk
-//               async copies (cp.async.bulk, completion on mbarriers).
-// Compute warps pack a tile into a shared-memory staging buffer at
-// tile-local offsets, then, while the look-back of that tile resolves,
-// compute the next tile; the staged words are copied to their final global
-// position one tile later.  Every wait is bounded (kErrTimeout), every global
-// store is checked against the caller's capacity (kErrCapacity).
+// CTA organisation (352 threads, 2 CTAs per SM, cooperative persistent grid;
+// tile t = chunk t of 4096 elements is processed by CTA t mod gridDim.x):
+//   warps 0..7   compute: each owns a contiguous 512-element slice of the
+//                tile, held as warp-tiles of 32*V elements (V = 8 consecutive
+//                elements per lane); a block of B elements spans LPB = B/V
+//                lanes.  A warp packs its slice
+//                into its own shared-memory ring (sized for typical packed
+//                output, not the worst case) and releases the input stage at
+//                once; the last warp to finish a tile publishes the tile's
+//                aggregate (record words, outliers).  Packed words are copied
+//                to their final position once the tile's prefix is known,
+//                up to kD - 1 tiles later, so look-back latency overlaps with
+//                the compute of later tiles.
+//   warps 8, 9   look-back (CTA tile iterations i with i mod 2 = warp - 8):
+//                resolve the exclusive prefix of a tile from the
+//                predecessors' status words (256 per L2 round trip), publish
+//                its inclusive prefix, write the chunk index entry (and the
+//                header for the last tile).
+//   warp 10      producer: streams the CTA's tiles into a 3-stage shared-
+//                memory ring with bulk async copies (cp.async.bulk,
+//                completion on mbarriers).
+// Every wait is bounded (kErrTimeout); every global store is checked against
+// the caller's capacity (kErrCapacity).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -37,21 +43,30 @@ namespace eblc {
 namespace {
 
 constexpr int kNW = 8;                    // compute warps
-constexpr int kS = 4;                     // input stages
-constexpr int kLookbackWarp = kNW;
-constexpr int kThreads = (kNW + 2) * 32;
+constexpr int kS = 3;                     // input stages
+constexpr int kD = 8;                     // tile slots: at most kD - 1 tiles computed but not finished
+constexpr int kLookbackWarps = 2;
+constexpr int kProducerWarp = kNW + kLookbackWarps;
+constexpr int kThreads = (kNW + kLookbackWarps + 1) * 32;
+constexpr int kWindow = 8;                // look-back status words per lane per round trip
+constexpr uint32_t kRing = 1536;          // packed words a compute warp can hold (3 worst-case tiles)
+constexpr uint32_t kWarpMax = kChunk / kNW;  // most words a warp packs for one tile
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint64_t kInclBit = 1ull << 63;
 
 struct __align__(128) EncSmem {
     float in[kS][kChunk];                 // input ring (bulk-copy destination)
-    uint32_t out[2][kChunk];              // packed payload staging, double buffered
-    uint8_t width[2][kChunk / 32];        // width bytes of the tile's blocks
-    uint32_t totals[2][kNW][2];           // per warp: payload words, outliers
-    uint32_t wprefix[2][kNW][2];          // per warp: exclusive prefix within the tile
-    uint32_t info[2][4];                  // record word offset, payload words, outliers, tile
+    uint32_t ring[kNW][kRing];            // per compute warp: packed words awaiting their prefix
+    uint32_t omask[kD][kNW][32];          // per slot, warp, lane: outlier bits
+    uint8_t width[kD][kChunk / 32];       // per slot: width bytes of the tile's blocks
+    uint32_t totals[kD][kNW][2];          // per slot, warp: payload words, outliers
+    uint32_t ringpos[kD][kNW];            // per slot, warp: ring offset of the packed words
+    int32_t slot_tile[kD];                // tile of the slot, -1 once the CTA has no more tiles
+    uint32_t done[kD];                    // CTA iteration + 1 once the slot's tile is written out
+    unsigned long long agg[kD];           // tile aggregate being summed: payload words | outliers << 32
+    uint32_t agg_count[kD];               // compute warps that have added to agg
     int32_t tile_id[kS];
-    uint64_t full[kS], empty[kS], computed[2], ready[2];
+    uint64_t full[kS], empty[kS], computed[kD];
     Bound bound;
 };
 
@@ -78,82 +93,50 @@ __device__ __forceinline__ uint32_t group_or(uint32_t v, int g) {
 
 __host__ __device__ constexpr int ilog2(int v) { return v <= 1 ? 0 : 1 + ilog2(v / 2); }
 
+
 // Pack the lane's V codes (width w, uniform over the lane's group of LPB
-// lanes) into the block's word array `dst` (shared memory): code j of the
-// block occupies bits [j*w, j*w + w), least significant bit first.  Lane r
-// of the group owns bits [r*V*w, (r+1)*V*w).  Lanes whose segment is
-// shorter than 32 bits are first merged pairwise (shuffles) until each
-// active lane holds at least 32 bits; then each word is shared by at most
-// two neighbouring segments, and the earlier lane's spill word is OR-ed into
-// the later lane's first word.
-template <int V, int LPB>
-__device__ __forceinline__ void pack_block(const uint32_t (&z)[V], uint32_t w, int r, int ln, uint32_t *dst) {
-    const uint32_t L = V * w;
-    uint32_t S[V + 1];
+// lanes) into the block's words at `dst` (shared memory, already zeroed):
+// code j of the block occupies bits [j*w, j*w + w), least significant bit
+// first.  Lane r of the group owns bits [r*V*w, (r+1)*V*w): it assembles
+// them in registers (NW words hold V*w bits for every width in the warp),
+// shifts them to their word alignment and ORs them in.  Neighbouring lanes
+// that share a word both OR into it, so no lane needs another lane's bits.
+template <int V, int NW>
+__device__ __forceinline__ void pack_lane(const uint32_t (&z)[V], uint32_t w, int r, uint32_t *dst) {
+    uint32_t S[NW + 1];
     S[0] = z[V - 1];
 #pragma unroll
-    for (int j = 1; j <= V; ++j) S[j] = 0u;
+    for (int j = 1; j <= NW; ++j) S[j] = 0u;
 #pragma unroll
     for (int v = V - 2; v >= 0; --v) {
 #pragma unroll
-        for (int j = V - 1 - v; j >= 1; --j) S[j] = __funnelshift_lc(S[j - 1], S[j], w);
+        for (int j = (V - 1 - v < NW - 1 ? V - 1 - v : NW - 1); j >= 1; --j)
+            S[j] = __funnelshift_lc(S[j - 1], S[j], w);
         S[0] = __funnelshift_lc(0u, S[0], w) | z[v];
     }
-
-    uint32_t Lc = L;
-    int stride = 1;
-    const bool short_seg = (w != 0u) && (L < 32u);
-    if (__any_sync(kFull, short_seg)) {
-        constexpr int kIters = ilog2(LPB) < ilog2(32 / V) ? ilog2(LPB) : ilog2(32 / V);
+    const uint32_t P = (uint32_t)r * V * w;  // bit offset of the segment in the block
+    const uint32_t s = P & 31u;
 #pragma unroll
-        for (int it = 0; it < kIters; ++it) {
-            const uint32_t o0 = __shfl_down_sync(kFull, S[0], 1 << it);
-            const uint32_t o1 = __shfl_down_sync(kFull, S[1], 1 << it);
-            if (short_seg && Lc < 32u) {
-                if ((r & ((2 << it) - 1)) == 0) {
-                    S[1] |= __funnelshift_lc(o0, o1, Lc);
-                    S[0] |= o0 << Lc;
-                }
-                Lc <<= 1;
-                stride <<= 1;
-            }
-        }
-    }
-    const bool active = (r & (stride - 1)) == 0;
-
-    const uint32_t P = (uint32_t)r * L;  // bit offset of the segment in the block
-    const uint32_t s = P & 31u, k0 = P >> 5;
-#pragma unroll
-    for (int j = V; j >= 1; --j) S[j] = __funnelshift_lc(S[j - 1], S[j], s);
+    for (int j = NW; j >= 1; --j) S[j] = __funnelshift_lc(S[j - 1], S[j], s);
     S[0] <<= s;
-    const uint32_t nw = (s + Lc + 31u) >> 5;
-    uint32_t last = S[0];
+    const uint32_t nw = (s + V * w + 31u) >> 5;
+    uint32_t *d = dst + (P >> 5);
 #pragma unroll
-    for (int j = 1; j <= V; ++j)
-        if (nw == (uint32_t)j + 1u) last = S[j];
-    const int src = (r >= stride) ? ln - stride : ln;
-    const uint32_t from_prev = __shfl_sync(kFull, last, src);
-    if (r >= stride && s != 0u) S[0] |= from_prev;
-    const bool last_shared = (r + stride < LPB) && (((P + Lc) & 31u) != 0u);
-    const uint32_t nstore = nw - (last_shared ? 1u : 0u);
-    if (active && w != 0u) {
-#pragma unroll
-        for (int j = 0; j <= V; ++j)
-            if ((uint32_t)j < nstore) dst[k0 + j] = S[j];
-    }
+    for (int j = 0; j <= NW; ++j)
+        if ((uint32_t)j < nw) atomicOr(d + j, S[j]);
 }
 
-// Quantize, test, delta, zigzag and pack one 4096-element tile held in
-// input stage s; packed words go to out[p] in this warp's region.
+// Quantize, test, delta, zigzag and pack this warp's slice of the tile in
+// input stage s; packed words go to `out` (this warp's ring, room for
+// kWarpMax words), width bytes to slot q.
 template <int V, int LPB>
-__device__ __forceinline__ void compute_tile(EncSmem &sm, const Bound &bd, int s, int p, uint32_t valid, int cw,
-                                             int ln, uint32_t &words_out, uint32_t &omask_out) {
+__device__ __forceinline__ void compute_tile(EncSmem &sm, const Bound &bd, int s, int q, uint32_t valid, int cw,
+                                             int ln, uint32_t *out, uint32_t &words_out, uint32_t &omask_out) {
     constexpr int kB = V * LPB;
     constexpr int kWT = 32 * V;
     constexpr int kWPW = kChunk / kWT / kNW;
     constexpr int kGroups = 32 / LPB;
     const int g = ln / LPB, r = ln % LPB;
-    uint32_t *region = sm.out[p] + cw * (kWPW * kWT);
     uint32_t wo = 0, omask = 0;
 
 #pragma unroll 1
@@ -172,48 +155,49 @@ __device__ __forceinline__ void compute_tile(EncSmem &sm, const Bound &bd, int s
         const uint32_t blk = (uint32_t)(wt * kWT) / kB + g;  // block index within the chunk
         const int cnt = min(max((int)valid - (int)(blk * kB), 0), kB);
 
-        int32_t q[V];
-        uint32_t obits = 0, abits = 0;
+        int32_t q_[V];
+        bool flagged = false;  // some element is not certainly within the bound
 #pragma unroll
         for (int v = 0; v < V; ++v) {
             const float y = __fmul_rn(x[v], bd.inv2eb);
             const int32_t qq = (fabsf(y) < 0x1p30f) ? __float2int_rn(y) : 0;
             const float xr = __fmul_rn(__int2float_rn(qq), bd.step);
-            const float d = fabsf(__fsub_rn(x[v], xr));
-            const bool out = d > bd.t_out;
-            const bool amb = !(d <= bd.t_in) && !out;
-            q[v] = qq;
-            obits |= (uint32_t)out << v;
-            abits |= (uint32_t)amb << v;
+            flagged |= !(fabsf(__fsub_rn(x[v], xr)) <= bd.t_in);
+            q_[v] = qq;
         }
+        uint32_t vm = (1u << V) - 1u;  // elements of this lane that exist
         if (valid < kChunk) {  // ragged last tile: elements at or beyond `valid` do not exist
             const uint32_t have = (e0 >= valid) ? 0u : min(valid - e0, (uint32_t)V);
-            const uint32_t vm = (have >= 32u) ? kFull : ((1u << have) - 1u);
+            vm = (1u << have) - 1u;
 #pragma unroll
             for (int v = 0; v < V; ++v)
-                if (!((vm >> v) & 1u)) q[v] = 0;
-            obits &= vm;
-            abits &= vm;
+                if (!((vm >> v) & 1u)) q_[v] = 0;
         }
-        if (__any_sync(kFull, abits != 0u)) {  // fp64 bound test where the fp32 filter is undecided
+        uint32_t obits = 0;
+        if (__any_sync(kFull, flagged)) {
+            // Outlier test proper: certainly out beyond t_out, fp64 test in the
+            // band between the fp32 filter thresholds (and for NaN).
 #pragma unroll
             for (int v = 0; v < V; ++v) {
-                if ((abits >> v) & 1u) {
-                    const float xr = __fmul_rn(__int2float_rn(q[v]), bd.step);
+                const float xr = __fmul_rn(__int2float_rn(q_[v]), bd.step);
+                const float d = fabsf(__fsub_rn(x[v], xr));
+                bool out = d > bd.t_out;
+                if (!out && !(d <= bd.t_in)) {
                     const bool finite = fabsf(x[v]) < __int_as_float(0x7f800000);
-                    const bool ok = fabs(__dsub_rn((double)x[v], (double)xr)) <= bd.eb;
-                    obits |= (uint32_t)(!finite || !ok) << v;
+                    out = !finite || !(fabs(__dsub_rn((double)x[v], (double)xr)) <= bd.eb);
                 }
+                obits |= (uint32_t)out << v;
             }
+            obits &= vm;
         }
 
-        int32_t pv = __shfl_up_sync(kFull, q[V - 1], 1);
+        int32_t pv = __shfl_up_sync(kFull, q_[V - 1], 1);
         if (r == 0) pv = 0;  // Lorenzo predecessor resets at the block start
         uint32_t z[V];
         uint32_t orz = 0;
 #pragma unroll
         for (int v = 0; v < V; ++v) {
-            const int32_t d = q[v] - (v ? q[v - 1] : pv);
+            const int32_t d = q_[v] - (v ? q_[v - 1] : pv);
             z[v] = ((uint32_t)d << 1) ^ (uint32_t)(d >> 31);
         }
         if (valid < kChunk) {
@@ -232,8 +216,20 @@ __device__ __forceinline__ void compute_tile(EncSmem &sm, const Bound &bd, int s
             pre += (gg < g) ? b : 0u;
             tot += b;
         }
-        if (r == 0) sm.width[p][blk] = (uint8_t)w;
-        pack_block<V, LPB>(z, w, r, ln, region + wo + pre);
+        if (r == 0) sm.width[q][blk] = (uint8_t)w;
+        uint32_t *o = out + wo;
+        for (uint32_t j = ln; j < tot; j += 32) o[j] = 0u;
+        __syncwarp();
+        const uint32_t wmax = __reduce_max_sync(kFull, w);
+        if (w != 0u) {
+            if (wmax * V <= 32u)
+                pack_lane<V, 1>(z, w, r, o + pre);
+            else if (wmax * V <= 96u)
+                pack_lane<V, 3>(z, w, r, o + pre);
+            else
+                pack_lane<V, V>(z, w, r, o + pre);
+        }
+        __syncwarp();
         wo += tot;
         omask |= obits << (k * V);
     }
@@ -241,110 +237,177 @@ __device__ __forceinline__ void compute_tile(EncSmem &sm, const Bound &bd, int s
     omask_out = omask;
 }
 
-// Copy one finished tile of this warp to its final position: payload words,
-// outliers (indices then values after the tile's payload), widths.
-template <int V, int LPB>
-__device__ __forceinline__ bool finish_tile(EncSmem &sm, const EncodeArgs &a, const Layout &L, uint32_t iprev,
-                                            int tile, int stage, uint32_t words, uint32_t omask, int cw, int ln) {
-    constexpr int kB = V * LPB;
-    constexpr int kWT = 32 * V;
-    constexpr int kWPW = kChunk / kWT / kNW;
-    const int q = iprev & 1;
-    if (!mbar_wait(&sm.ready[q], (iprev >> 1) & 1, a.wait_ns, a.err)) return false;
-    const uint32_t rec = sm.info[q][0], PW = sm.info[q][1], MT = sm.info[q][2];
-    const uint32_t wpw = sm.wprefix[q][cw][0], wpo = sm.wprefix[q][cw][1];
-    uint32_t *recs = reinterpret_cast<uint32_t *>(a.out + L.record_off);
-    const uint64_t cap_words = (a.out_cap > L.record_off) ? (a.out_cap - L.record_off) / 4 : 0;
-    bool over = false;
-
-    const uint32_t *src = sm.out[q] + cw * (kWPW * kWT);
-    const uint64_t w0 = (uint64_t)rec + wpw;
-    for (uint32_t j = ln; j < words; j += 32) {
-        if (w0 + j < cap_words)
-            st_cs_u32(recs + w0 + j, src[j]);
-        else
-            over = true;
-    }
-
-    if (__any_sync(kFull, omask != 0u)) {
-        uint32_t ord_base = 0;
-#pragma unroll 1
-        for (int k = 0; k < kWPW; ++k) {
-            uint32_t bits = (omask >> (k * V)) & ((1u << V) - 1u);
-            const uint32_t c = __popc(bits);
-            uint32_t incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t t = __shfl_up_sync(kFull, incl, o);
-                if (ln >= o) incl += t;
-            }
-            uint32_t ord = ord_base + incl - c;
-            while (bits) {
-                const int v = __ffs(bits) - 1;
-                bits &= bits - 1u;
-                const uint32_t e = (uint32_t)(cw * kWPW + k) * kWT + ln * V + v;
-                const uint64_t pi = (uint64_t)rec + PW + wpo + ord;
-                const uint64_t pv = pi + MT;
-                if (pv < cap_words) {
-                    recs[pi] = (uint32_t)tile * kChunk + e;
-                    recs[pv] = __float_as_uint(sm.in[stage][e]);
-                } else {
-                    over = true;
-                }
-                ++ord;
-            }
-            ord_base += __shfl_sync(kFull, incl, 31);
-        }
-    }
-
-    {  // this warp's width bytes (zeros past the last block up to the 16-byte pad)
-        constexpr uint32_t kBPW = kChunk / kB / kNW;  // blocks per warp per tile
-        const uint64_t b = (uint64_t)tile * (kChunk / kB) + cw * kBPW + ln;
-        const uint64_t off = L.width_off + b;
-        if (ln < (int)kBPW && b < pad16(L.nb)) {
-            if (off < a.out_cap)
-                a.out[off] = sm.width[q][cw * kBPW + ln];
-            else
-                over = true;
-        }
-    }
-    if (__any_sync(kFull, over) && ln == 0) atomicOr(a.err, kErrCapacity);
-    __syncwarp();
-    if (ln == 0) mbar_arrive(&sm.empty[stage]);
-    return true;
+__device__ __forceinline__ bool slot_done(const EncSmem &sm, uint32_t it) {
+    return *reinterpret_cast<const volatile uint32_t *>(&sm.done[it % kD]) == it + 1;
 }
 
 template <int V, int LPB>
-__device__ void compute_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L, int cw, int ln) {
+__device__ void compute_warp(EncSmem &sm, const EncodeArgs &a, int cw, int ln) {
     const Bound bd = sm.bound;
-    int prev_tile = -1, prev_stage = 0;
-    uint32_t prev_words = 0, prev_omask = 0;
+    uint32_t *ring = sm.ring[cw];
+    uint32_t oldest = 0;  // oldest CTA iteration whose packed words still occupy this warp's ring
+    uint32_t head = 0;    // ring offset after the newest tile's words
     uint32_t i = 0;
+    uint64_t t0 = 0;
     for (;; ++i) {
-        const int s = i % kS, p = i & 1;
+        // Reclaim ring space of tiles already written out, then find room for a
+        // worst-case tile: a free slot and kWarpMax contiguous ring words.
+        uint32_t start = 0;
+        for (;;) {
+            while (oldest < i && slot_done(sm, oldest)) ++oldest;
+            if (i - oldest <= (uint32_t)kD - 2) {
+                if (oldest == i) {
+                    start = 0;
+                    break;
+                }
+                const uint32_t tail = sm.ringpos[oldest % kD][cw];
+                if (head >= tail) {
+                    if (head + kWarpMax <= kRing) { start = head; break; }
+                    if (kWarpMax <= tail) { start = 0; break; }
+                } else if (head + kWarpMax <= tail) {
+                    start = head;
+                    break;
+                }
+            }
+            if (t0 == 0) t0 = globaltimer_ns();
+            if (globaltimer_ns() - t0 > a.wait_ns) {
+                if (ln == 0) atomicOr(a.err, kErrTimeout);
+                return;
+            }
+            __nanosleep(64);
+        }
+        t0 = 0;
+        const int s = i % kS, q = i % kD;
         if (!mbar_wait(&sm.full[s], (i / kS) & 1, a.wait_ns, a.err)) return;
         const int tile = sm.tile_id[s];
         if (tile < 0) break;
         const uint64_t e0 = (uint64_t)tile * kChunk;
         const uint32_t valid = (uint32_t)min((uint64_t)kChunk, a.n - e0);
         uint32_t words, omask;
-        compute_tile<V, LPB>(sm, bd, s, p, valid, cw, ln, words, omask);
+        compute_tile<V, LPB>(sm, bd, s, q, valid, cw, ln, ring + start, words, omask);
         const uint32_t outl = __reduce_add_sync(kFull, __popc(omask));
-        if (ln == 0) {
-            sm.totals[p][cw][0] = words;
-            sm.totals[p][cw][1] = outl;
-        }
+        sm.omask[q][cw][ln] = omask;
         __syncwarp();
-        if (ln == 0) mbar_arrive(&sm.computed[p]);
-        if (prev_tile >= 0 &&
-            !finish_tile<V, LPB>(sm, a, L, i - 1, prev_tile, prev_stage, prev_words, prev_omask, cw, ln))
-            return;
-        prev_tile = tile;
-        prev_stage = s;
-        prev_words = words;
-        prev_omask = omask;
+        if (ln == 0) {
+            mbar_arrive(&sm.empty[s]);  // the input stage is free again
+            sm.totals[q][cw][0] = words;
+            sm.totals[q][cw][1] = outl;
+            sm.ringpos[q][cw] = start;
+            if (cw == 0) sm.slot_tile[q] = tile;
+            // The last warp to finish the tile publishes its aggregate at once, so
+            // successors' look-backs never wait for this CTA's look-back warps.
+            atomicAdd(&sm.agg[q], (unsigned long long)words | ((unsigned long long)outl << 32));
+            __threadfence_block();
+            if (atomicAdd(&sm.agg_count[q], 1u) == kNW - 1) {
+                __threadfence_block();
+                const unsigned long long t = atomicExch(&sm.agg[q], 0ull);
+                sm.agg_count[q] = 0;
+                const uint32_t PW = (uint32_t)t, MT = (uint32_t)(t >> 32);
+                if (tile != a.stall_tile)
+                    st_relaxed_gpu(&a.status[tile], pack_status(PW + 2u * MT, MT, tile == 0));
+            }
+            mbar_arrive(&sm.computed[q]);
+        }
+        head = start + words;
     }
-    if (prev_tile >= 0) finish_tile<V, LPB>(sm, a, L, i - 1, prev_tile, prev_stage, prev_words, prev_omask, cw, ln);
+    // Tell both look-back warps that this CTA has no more tiles: iterations i
+    // and i + 1 get tile -1.  Their slots must be free of pending tiles first.
+    while (i - oldest > (uint32_t)(kD - kLookbackWarps)) {
+        if (!slot_done(sm, oldest)) {
+            if (t0 == 0) t0 = globaltimer_ns();
+            if (globaltimer_ns() - t0 > a.wait_ns) {
+                if (ln == 0) atomicOr(a.err, kErrTimeout);
+                return;
+            }
+            __nanosleep(64);
+            continue;
+        }
+        ++oldest;
+    }
+    if (ln == 0) {
+        if (cw == 0)
+            for (int j = 0; j < kLookbackWarps; ++j) sm.slot_tile[(i + j) % kD] = -1;
+        __threadfence_block();
+        for (int j = 0; j < kLookbackWarps; ++j) mbar_arrive(&sm.computed[(i + j) % kD]);
+    }
+}
+
+// Write the tile of CTA iteration `it` (slot q) to its final position once
+// its prefix (record word offset rec, payload words PW, outliers MT) is
+// known: every compute warp's packed words from its ring, the outliers
+// (indices then values after the tile's payload; values read back from the
+// input array) and the width bytes.  Lane c < kNW of this warp holds compute
+// warp c's exclusive prefix (words wpw, outliers wpo) within the tile.
+template <int V, int LPB>
+__device__ __forceinline__ void write_tile(EncSmem &sm, const EncodeArgs &a, const Layout &L, int q, int tile,
+                                           uint32_t rec, uint32_t PW, uint32_t MT, uint32_t wpw, uint32_t wpo,
+                                           int ln) {
+    constexpr int kB = V * LPB;
+    constexpr int kWT = 32 * V;
+    constexpr int kWPW = kChunk / kWT / kNW;
+    uint32_t *recs = reinterpret_cast<uint32_t *>(a.out + L.record_off);
+    const uint64_t cap_words = (a.out_cap > L.record_off) ? (a.out_cap - L.record_off) / 4 : 0;
+    bool over = false;
+    const float *xin = a.in + (uint64_t)tile * kChunk;
+#pragma unroll 1
+    for (int c = 0; c < kNW; ++c) {
+        const uint32_t words = sm.totals[q][c][0], pos = sm.ringpos[q][c];
+        const uint64_t w0 = (uint64_t)rec + __shfl_sync(kFull, wpw, c);
+        const uint32_t *src = sm.ring[c] + pos;
+        for (uint32_t j = ln; j < words; j += 32) {
+            if (w0 + j < cap_words)
+                st_cs_u32(recs + w0 + j, src[j]);
+            else
+                over = true;
+        }
+        const uint32_t omask = sm.omask[q][c][ln];
+        const uint32_t obase = __shfl_sync(kFull, wpo, c);
+        if (__any_sync(kFull, omask != 0u)) {
+            uint32_t ord_base = 0;
+#pragma unroll 1
+            for (int k = 0; k < kWPW; ++k) {
+                uint32_t bits = (omask >> (k * V)) & ((1u << V) - 1u);
+                const uint32_t cnt = __popc(bits);
+                uint32_t incl = cnt;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t t = __shfl_up_sync(kFull, incl, o);
+                    if (ln >= o) incl += t;
+                }
+                uint32_t ord = ord_base + incl - cnt;
+                while (bits) {
+                    const int v = __ffs(bits) - 1;
+                    bits &= bits - 1u;
+                    const uint32_t e = (uint32_t)(c * kWPW + k) * kWT + ln * V + v;
+                    const uint64_t pi = (uint64_t)rec + PW + obase + ord;
+                    const uint64_t pv = pi + MT;
+                    if (pv < cap_words) {
+                        recs[pi] = (uint32_t)tile * kChunk + e;
+                        recs[pv] = __float_as_uint(__ldg(xin + e));
+                    } else {
+                        over = true;
+                    }
+                    ++ord;
+                }
+                ord_base += __shfl_sync(kFull, incl, 31);
+            }
+        }
+    }
+    {  // width bytes of the tile's blocks, zeros past the last block up to the 16-byte pad
+        constexpr uint32_t K = kChunk / kB;
+        const uint64_t b0 = (uint64_t)tile * K;
+        const uint64_t bend = min(b0 + K, pad16(L.nb));
+        const uint32_t nwords = (uint32_t)((bend - b0) / 4);
+        const uint32_t *ws = reinterpret_cast<const uint32_t *>(sm.width[q]);
+        uint32_t *wd = reinterpret_cast<uint32_t *>(a.out + L.width_off + b0);
+        for (uint32_t j = ln; j < nwords; j += 32) {
+            if (L.width_off + b0 + 4 * j + 4 <= a.out_cap)
+                wd[j] = ws[j];
+            else
+                over = true;
+        }
+    }
+    if (__any_sync(kFull, over) && ln == 0) atomicOr(a.err, kErrCapacity);
 }
 
 __device__ void write_header(const EncodeArgs &a, const Layout &L, const Bound &bd, uint64_t R, uint64_t m) {
@@ -396,16 +459,85 @@ __device__ void write_header(const EncodeArgs &a, const Layout &L, const Bound &
         *reinterpret_cast<uint32_t *>(a.out + b) = 0u;
 }
 
-__device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L, int ln) {
-    for (uint32_t i = 0;; ++i) {
-        const int s = i % kS, p = i & 1;
-        if (!mbar_wait(&sm.full[s], (i / kS) & 1, a.wait_ns, a.err)) return;
-        const int tile = sm.tile_id[s];
-        if (tile < 0) break;
-        if (!mbar_wait(&sm.computed[p], (i >> 1) & 1, a.wait_ns, a.err)) return;
+// Exclusive prefix (record words, outliers) of `tile` from its predecessors'
+// status words: each lane reads kWindow consecutive predecessors, so one L2
+// round trip covers 32 * kWindow tiles.  Stops at the nearest inclusive
+// prefix; every tile between it and `tile` must have published at least its
+// aggregate (spins with back-off until they have, bounded by wait_ns).
+__device__ __forceinline__ void look_back(const EncodeArgs &a, int tile, int ln, uint32_t &exR, uint32_t &exM) {
+    exR = 0;
+    exM = 0;
+    int64_t base = (int64_t)tile - 1;
+    uint64_t t0 = 0;
+    uint32_t backoff = 32;
+    while (base >= 0) {
+        uint64_t v[kWindow];
+#pragma unroll
+        for (int j = 0; j < kWindow; ++j) {
+            const int64_t pi = base - (int64_t)ln * kWindow - j;
+            v[j] = (pi >= 0) ? ld_relaxed_gpu(&a.status[pi]) : pack_status(0, 0, true);
+        }
+        int first_incl = kWindow;
+        bool missing = false;
+#pragma unroll
+        for (int j = kWindow - 1; j >= 0; --j)
+            if (v[j] & kInclBit) first_incl = j;
+#pragma unroll
+        for (int j = 0; j < kWindow; ++j)
+            if (j < first_incl && v[j] == 0) missing = true;
+        const uint32_t im = __ballot_sync(kFull, first_incl < kWindow);
+        const int J = im ? __ffs(im) - 1 : 32;  // first lane holding an inclusive prefix
+        const uint32_t miss = __ballot_sync(kFull, ln <= J && missing);
+        if (miss) {
+            // Wait on the nearest predecessor that has published nothing yet,
+            // polling that one word only, then read the window again.
+            int jm = kWindow;
+#pragma unroll
+            for (int j = kWindow - 1; j >= 0; --j)
+                if (j < first_incl && v[j] == 0) jm = j;
+            const int lm = __ffs(miss) - 1;
+            const int jw = __shfl_sync(kFull, jm, lm);
+            const uint64_t *w = &a.status[base - (int64_t)lm * kWindow - jw];
+            if (t0 == 0) t0 = globaltimer_ns();
+            while (ld_relaxed_gpu(w) == 0) {
+                if (globaltimer_ns() - t0 > a.wait_ns) {  // give up: record and move on
+                    if (ln == 0) atomicOr(a.err, kErrTimeout);
+                    return;
+                }
+                __nanosleep(backoff);
+                backoff = min(backoff * 2u, 512u);
+            }
+            __syncwarp();
+            continue;
+        }
+        uint32_t sr = 0, sm_ = 0;
+        if (ln <= J) {
+            const int upto = (ln < J) ? kWindow - 1 : first_incl;
+#pragma unroll
+            for (int j = 0; j < kWindow; ++j) {
+                if (j <= upto) {
+                    sr += (uint32_t)(v[j] & 0xffffffffu) - 1u;
+                    sm_ += (uint32_t)((v[j] >> 32) & 0x7fffffffu);
+                }
+            }
+        }
+        exR += __reduce_add_sync(kFull, sr);
+        exM += __reduce_add_sync(kFull, sm_);
+        if (J < 32) return;
+        base -= 32 * kWindow;
+    }
+}
 
-        const uint32_t tw = (ln < kNW) ? sm.totals[p][ln][0] : 0u;
-        const uint32_t to = (ln < kNW) ? sm.totals[p][ln][1] : 0u;
+template <int V, int LPB>
+__device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L, int lw, int ln) {
+    for (uint32_t i = lw;; i += kLookbackWarps) {
+        const int q = i % kD;
+        if (!mbar_wait(&sm.computed[q], (i / kD) & 1, a.wait_ns, a.err)) return;
+        const int tile = sm.slot_tile[q];
+        if (tile < 0) break;
+
+        const uint32_t tw = (ln < kNW) ? sm.totals[q][ln][0] : 0u;
+        const uint32_t to = (ln < kNW) ? sm.totals[q][ln][1] : 0u;
         uint32_t iw = tw, io = to;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -417,54 +549,19 @@ __device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
             }
         }
         const uint32_t PW = __shfl_sync(kFull, iw, 31), MT = __shfl_sync(kFull, io, 31);
-        if (ln < kNW) {
-            sm.wprefix[p][ln][0] = iw - tw;
-            sm.wprefix[p][ln][1] = io - to;
-        }
         const uint32_t Rt = PW + 2u * MT;
         const bool publish = (tile != a.stall_tile);
 
         uint32_t exR = 0, exM = 0;
-        if (tile == 0) {
-            if (ln == 0 && publish) st_relaxed_gpu(&a.status[0], pack_status(Rt, MT, true));
-        } else {
-            if (ln == 0 && publish) st_relaxed_gpu(&a.status[tile], pack_status(Rt, MT, false));
-            int64_t base = tile - 1;
-            uint64_t t0 = 0;
-            uint32_t backoff = 32;
-            for (;;) {
-                const int64_t pi = base - ln;
-                const uint64_t v = (pi >= 0) ? ld_relaxed_gpu(&a.status[pi]) : pack_status(0, 0, true);
-                const uint32_t incl_mask = __ballot_sync(kFull, (v & kInclBit) != 0);
-                const uint32_t none_mask = __ballot_sync(kFull, v == 0);
-                const int J = incl_mask ? __ffs(incl_mask) - 1 : 32;
-                const uint32_t below = (J == 32) ? kFull : ((1u << J) - 1u);
-                if (none_mask & below) {
-                    if (t0 == 0) t0 = globaltimer_ns();
-                    if (globaltimer_ns() - t0 > a.wait_ns) {  // give up: record and move on
-                        if (ln == 0) atomicOr(a.err, kErrTimeout);
-                        break;
-                    }
-                    __nanosleep(backoff);
-                    backoff = min(backoff * 2u, 1024u);
-                    continue;
-                }
-                const bool take = (ln <= J);
-                const uint32_t vr = take ? (uint32_t)(v & 0xffffffffu) - 1u : 0u;
-                const uint32_t vm = take ? (uint32_t)((v >> 32) & 0x7fffffffu) : 0u;
-                exR += __reduce_add_sync(kFull, vr);
-                exM += __reduce_add_sync(kFull, vm);
-                if (J < 32) break;
-                base -= 32;
-            }
+        if (tile != 0) {  // the aggregate is already published by the compute warps
+            // Start once this CTA has also computed its next tile: by then the
+            // other CTAs have almost always published this tile's predecessors
+            // of the same wave, so the look-back rarely has to wait.
+            if (!mbar_wait(&sm.computed[(i + 1) % kD], ((i + 1) / kD) & 1, a.wait_ns, a.err)) return;
+            look_back(a, tile, ln, exR, exM);
             if (ln == 0 && publish) st_relaxed_gpu(&a.status[tile], pack_status(exR + Rt, exM + MT, true));
         }
-
         if (ln == 0) {
-            sm.info[p][0] = exR;
-            sm.info[p][1] = PW;
-            sm.info[p][2] = MT;
-            sm.info[p][3] = (uint32_t)tile;
             a.status_next[tile] = 0ull;
             const uint64_t io_off = L.index_off + 8ull * (uint64_t)tile;
             if (io_off + 8 <= a.out_cap)
@@ -474,40 +571,42 @@ __device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
             if ((uint64_t)tile == L.nc - 1)
                 write_header(a, L, sm.bound, (uint64_t)exR + Rt, (uint64_t)exM + MT);
         }
+        write_tile<V, LPB>(sm, a, L, q, tile, exR, PW, MT, iw - tw, io - to, ln);
         __syncwarp();
-        if (ln == 0) mbar_arrive(&sm.ready[p]);
+        if (ln == 0) {
+            __threadfence_block();
+            *reinterpret_cast<volatile uint32_t *>(&sm.done[q]) = i + 1;
+        }
     }
 }
 
+// Tile t is processed by CTA t mod gridDim.x, in increasing t.  The grid is
+// launched cooperatively (all CTAs resident at once), so every tile a
+// look-back waits for belongs to a running CTA that reaches it without
+// waiting on anything later: the look-back cannot deadlock.
 __device__ void producer_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L, int ln) {
     if (ln != 0) return;
-    uint32_t issued = 0;  // stages with an outstanding fill
-    uint32_t next = atomicAdd(a.counter, 1u);
     uint32_t i = 0;
     for (;; ++i) {
         const int s = i % kS;
         if (i >= kS && !mbar_wait(&sm.empty[s], ((i / kS) - 1) & 1, a.wait_ns, a.err)) break;
-        const uint32_t t = next;
-        if ((uint64_t)t >= L.nc) {
+        const uint64_t t = (uint64_t)blockIdx.x + (uint64_t)i * gridDim.x;
+        if (t >= L.nc) {
             sm.tile_id[s] = -1;
             mbar_arrive(&sm.full[s]);
-            issued |= 1u << s;
             ++i;
             break;
         }
-        next = atomicAdd(a.counter, 1u);  // claim the following tile early
         sm.tile_id[s] = (int32_t)t;
-        const uint64_t e0 = (uint64_t)t * kChunk;
+        const uint64_t e0 = t * kChunk;
         const uint32_t valid = (uint32_t)min((uint64_t)kChunk, a.n - e0);
         const uint32_t bulk = (valid * 4u) & ~15u;
         for (uint32_t j = bulk / 4; j < valid; ++j) sm.in[s][j] = a.in[e0 + j];
         mbar_arrive_expect_tx(&sm.full[s], bulk);
         if (bulk) bulk_g2s(sm.in[s], a.in + e0, bulk, &sm.full[s]);
-        issued |= 1u << s;
     }
     // Drain: no copy into this CTA's shared memory may still be in flight at exit.
     for (int s = 0; s < kS; ++s) {
-        if (!((issued >> s) & 1u)) continue;
         const uint32_t uses = (i > (uint32_t)s) ? (i - 1 - s) / kS + 1 : 0;  // fills issued on stage s
         if (uses) mbar_wait(&sm.full[s], (uses - 1) & 1, a.wait_ns, a.err);
     }
@@ -525,9 +624,11 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const EncodeArgs a)
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kNW);
         }
-        for (int p = 0; p < 2; ++p) {
-            mbar_init(&sm.computed[p], kNW);
-            mbar_init(&sm.ready[p], 1);
+        for (int q = 0; q < kD; ++q) {
+            mbar_init(&sm.computed[q], kNW);
+            sm.done[q] = 0u;
+            sm.agg[q] = 0ull;
+            sm.agg_count[q] = 0u;
         }
         mbar_init_fence();
         const float vmin = a.abs_mode ? 0.0f : a.range[0];
@@ -541,9 +642,9 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const EncodeArgs a)
     __syncthreads();
 
     if (warp < kNW)
-        compute_warp<V, LPB>(sm, a, L, warp, ln);
-    else if (warp == kLookbackWarp)
-        lookback_warp(sm, a, L, ln);
+        compute_warp<V, LPB>(sm, a, warp, ln);
+    else if (warp < kProducerWarp)
+        lookback_warp<V, LPB>(sm, a, L, warp - kNW, ln);
     else
         producer_warp(sm, a, L, ln);
 
@@ -556,20 +657,26 @@ cudaError_t launch_t(const EncodeArgs &a, int num_sms, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(encode_kernel<V, LPB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_kernel<V, LPB>, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
     const Layout L = stream_layout(a.n, a.block);
-    const uint64_t want = (uint64_t)num_sms * 2;
-    const int grid = (int)(L.nc == 0 ? 1 : (want < L.nc ? want : L.nc));
-    encode_kernel<V, LPB><<<grid, kThreads, smem, stream>>>(a);
-    return cudaGetLastError();
+    const uint64_t resident = (uint64_t)per_sm * (uint64_t)num_sms;
+    const int grid = (int)(L.nc == 0 ? 1 : (resident < L.nc ? resident : L.nc));
+    EncodeArgs args = a;
+    void *params[] = {&args};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(encode_kernel<V, LPB>), dim3(grid),
+                                       dim3(kThreads), params, smem, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_encode(const EncodeArgs &a, int num_sms, cudaStream_t stream) {
     switch (a.block) {
-        case 32: return launch_t<4, 8>(a, num_sms, stream);
-        case 64: return launch_t<4, 16>(a, num_sms, stream);
-        case 128: return launch_t<4, 32>(a, num_sms, stream);
+        case 32: return launch_t<8, 4>(a, num_sms, stream);
+        case 64: return launch_t<8, 8>(a, num_sms, stream);
+        case 128: return launch_t<8, 16>(a, num_sms, stream);
         case 256: return launch_t<8, 32>(a, num_sms, stream);
         default: return cudaErrorInvalidValue;
     }
