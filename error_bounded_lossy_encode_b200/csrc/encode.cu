@@ -28,7 +28,7 @@
 //                the compute of later tiles.
 //   warps 8, 9   look-back (CTA tile iterations i with i mod 2 = warp - 8):
 //                resolve the exclusive prefix of a tile from the
-//                predecessors' status words (256 per L2 round trip), publish
+//                predecessors' status words (320 per coalesced L2 round trip), publish
 //                its inclusive prefix, write the chunk index entry (and the
 //                header for the last tile).
 //   warp 10      producer: streams the CTA's tiles into a 3-stage shared-
@@ -48,7 +48,7 @@ constexpr int kD = 8;                     // tile slots: at most kD - 1 tiles co
 constexpr int kLookbackWarps = 2;
 constexpr int kProducerWarp = kNW + kLookbackWarps;
 constexpr int kThreads = (kNW + kLookbackWarps + 1) * 32;
-constexpr int kWindow = 8;                // look-back status words per lane per round trip
+constexpr int kWindow = 10;               // look-back rows of 32 status words per round trip
 constexpr uint32_t kRing = 1536;          // packed words a compute warp can hold (3 worst-case tiles)
 constexpr uint32_t kWarpMax = kChunk / kNW;  // most words a warp packs for one tile
 constexpr uint32_t kFull = 0xffffffffu;
@@ -460,47 +460,56 @@ __device__ void write_header(const EncodeArgs &a, const Layout &L, const Bound &
 }
 
 // Exclusive prefix (record words, outliers) of `tile` from its predecessors'
-// status words: each lane reads kWindow consecutive predecessors, so one L2
-// round trip covers 32 * kWindow tiles.  Stops at the nearest inclusive
-// prefix; every tile between it and `tile` must have published at least its
-// aggregate (spins with back-off until they have, bounded by wait_ns).
-__device__ __forceinline__ void look_back(const EncodeArgs &a, int tile, int ln, uint32_t &exR, uint32_t &exM) {
+// status words, nearest first, stopping at the nearest inclusive prefix.
+// Tile `stop` (-1 before tile 0) is known to have the inclusive prefix
+// `known` (status word form), so no status word at or below it is read.  One
+// L2 round trip reads kWindow rows of 32 consecutive status words (row j,
+// lane l: predecessor tile - 1 - 32 j - l), coalesced.  Every tile between
+// the inclusive prefix found and `tile` must have published at least its
+// aggregate: polls the nearest missing one with back-off (bounded by
+// wait_ns, and given up at once when another wait of the launch has timed
+// out), then reads the window again.
+__device__ __forceinline__ void look_back(const EncodeArgs &a, int tile, int stop, uint64_t known, int ln,
+                                          uint32_t &exR, uint32_t &exM) {
     exR = 0;
     exM = 0;
-    int64_t base = (int64_t)tile - 1;
+    int base = tile - 1;  // nearest predecessor not yet summed
     uint64_t t0 = 0;
     uint32_t backoff = 32;
-    while (base >= 0) {
+    while (base > stop - 1) {
         uint64_t v[kWindow];
 #pragma unroll
         for (int j = 0; j < kWindow; ++j) {
-            const int64_t pi = base - (int64_t)ln * kWindow - j;
-            v[j] = (pi >= 0) ? ld_relaxed_gpu(&a.status[pi]) : pack_status(0, 0, true);
+            const int p = base - 32 * j - ln;
+            v[j] = (p > stop) ? ld_relaxed_gpu(&a.status[p]) : (p == stop ? known : pack_status(0, 0, true));
         }
-        int first_incl = kWindow;
-        bool missing = false;
+        uint32_t sr = 0, sm_ = 0;
+        int found = 0, miss_row = -1;
+        uint32_t miss_lanes = 0;
 #pragma unroll
-        for (int j = kWindow - 1; j >= 0; --j)
-            if (v[j] & kInclBit) first_incl = j;
-#pragma unroll
-        for (int j = 0; j < kWindow; ++j)
-            if (j < first_incl && v[j] == 0) missing = true;
-        const uint32_t im = __ballot_sync(kFull, first_incl < kWindow);
-        const int J = im ? __ffs(im) - 1 : 32;  // first lane holding an inclusive prefix
-        const uint32_t miss = __ballot_sync(kFull, ln <= J && missing);
-        if (miss) {
-            // Wait on the nearest predecessor that has published nothing yet,
-            // polling that one word only, then read the window again.
-            int jm = kWindow;
-#pragma unroll
-            for (int j = kWindow - 1; j >= 0; --j)
-                if (j < first_incl && v[j] == 0) jm = j;
-            const int lm = __ffs(miss) - 1;
-            const int jw = __shfl_sync(kFull, jm, lm);
-            const uint64_t *w = &a.status[base - (int64_t)lm * kWindow - jw];
+        for (int j = 0; j < kWindow; ++j) {
+            const uint32_t inc = __ballot_sync(kFull, (v[j] & kInclBit) != 0ull);
+            const uint32_t mis = __ballot_sync(kFull, v[j] == 0ull);
+            if (!found && miss_row < 0) {
+                const uint32_t upto = inc ? (inc ^ (inc - 1u)) : kFull;  // lanes through the first inclusive
+                if (mis & upto) {
+                    miss_row = j;
+                    miss_lanes = mis & upto;
+                } else {
+                    if ((upto >> ln) & 1u) {
+                        sr += (uint32_t)(v[j] & 0xffffffffu) - 1u;
+                        sm_ += (uint32_t)((v[j] >> 32) & 0x7fffffffu);
+                    }
+                    found = inc != 0u;
+                }
+            }
+        }
+        if (miss_row >= 0) {
+            const uint64_t *w = &a.status[base - 32 * miss_row - (__ffs(miss_lanes) - 1)];
             if (t0 == 0) t0 = globaltimer_ns();
             while (ld_relaxed_gpu(w) == 0) {
-                if (globaltimer_ns() - t0 > a.wait_ns) {  // give up: record and move on
+                if (globaltimer_ns() - t0 > a.wait_ns ||
+                    (*reinterpret_cast<volatile uint32_t *>(a.err) & kErrTimeout)) {  // give up: record, move on
                     if (ln == 0) atomicOr(a.err, kErrTimeout);
                     return;
                 }
@@ -510,20 +519,9 @@ __device__ __forceinline__ void look_back(const EncodeArgs &a, int tile, int ln,
             __syncwarp();
             continue;
         }
-        uint32_t sr = 0, sm_ = 0;
-        if (ln <= J) {
-            const int upto = (ln < J) ? kWindow - 1 : first_incl;
-#pragma unroll
-            for (int j = 0; j < kWindow; ++j) {
-                if (j <= upto) {
-                    sr += (uint32_t)(v[j] & 0xffffffffu) - 1u;
-                    sm_ += (uint32_t)((v[j] >> 32) & 0x7fffffffu);
-                }
-            }
-        }
         exR += __reduce_add_sync(kFull, sr);
         exM += __reduce_add_sync(kFull, sm_);
-        if (J < 32) return;
+        if (found) return;
         base -= 32 * kWindow;
     }
 }
@@ -558,7 +556,7 @@ __device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
             // other CTAs have almost always published this tile's predecessors
             // of the same wave, so the look-back rarely has to wait.
             if (!mbar_wait(&sm.computed[(i + 1) % kD], ((i + 1) / kD) & 1, a.wait_ns, a.err)) return;
-            look_back(a, tile, ln, exR, exM);
+            look_back(a, tile, -1, pack_status(0, 0, true), ln, exR, exM);
             if (ln == 0 && publish) st_relaxed_gpu(&a.status[tile], pack_status(exR + Rt, exM + MT, true));
         }
         if (ln == 0) {

@@ -268,8 +268,14 @@ eblc_status_t ensure_host_staging(eblc_plan_s *p) {
 }
 
 // Queue the compress kernels on `st` (device pointers).
-eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_in, uint8_t *d_out, uint64_t cap) {
-    timing_begin(p, st);
+// call_events: record the "call" timing pair around this enqueue (false when
+// the caller brackets a larger span, e.g. the HOST kind's copies).
+eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_in, uint8_t *d_out, uint64_t cap,
+                               bool call_events = true) {
+    if (call_events)
+        timing_begin(p, st);
+    else
+        p->timing.count = 0;
     const int par = p->parity;
     if (!p->abs_mode && p->n > 0) {
         RangeArgs ra{d_in, p->n, p->partials, p->range_counter, p->range};
@@ -302,7 +308,7 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
     timing_mark(p, st, false, nullptr);
     if (s != EBLC_OK) return s;
     s = cuda_status(cudaMemcpyAsync(p->h_rb, p->d_rb, sizeof(Readback), cudaMemcpyDeviceToHost, st), "readback");
-    timing_end(p, st);
+    if (call_events) timing_end(p, st);
     return s;
 }
 
@@ -538,20 +544,23 @@ EBLC_API eblc_status_t eblc_compress(eblc_plan_t p, const eblc_execution_t *exec
         if ((s = cuda_status(cudaStreamSynchronize(st), "compress sync")) != EBLC_OK) return s;
         return finish_compress(p, compressed_bytes, h_sidecar);
     }
-    // HOST: host pointers, same kernels on plan-owned device staging.
+    // HOST: host pointers, same kernels on plan-owned device staging.  The
+    // "call" timing pair spans the input copy through the stream copy back.
     if ((s = ensure_host_staging(p)) != EBLC_OK) return s;
     cudaStream_t st = p->host_stream;
     const uint64_t cap = std::min<uint64_t>(out_capacity, p->max_bytes);
+    timing_begin(p, st);
     if (p->n && (s = cuda_status(cudaMemcpyAsync(p->stage_in, d_in, 4 * p->n, cudaMemcpyHostToDevice, st), "h2d")) !=
                     EBLC_OK)
         return s;
-    if ((s = enqueue_compress(p, st, p->stage_in, p->stage_out, cap)) != EBLC_OK) return s;
+    if ((s = enqueue_compress(p, st, p->stage_in, p->stage_out, cap, false)) != EBLC_OK) return s;
     if ((s = cuda_status(cudaStreamSynchronize(st), "compress sync")) != EBLC_OK) return s;
     size_t total = 0;
     s = finish_compress(p, &total, h_sidecar);
     if (compressed_bytes) *compressed_bytes = total;
     if (s != EBLC_OK) return s;
     eblc_status_t c = cuda_status(cudaMemcpyAsync(d_out, p->stage_out, total, cudaMemcpyDeviceToHost, st), "d2h");
+    timing_end(p, st);
     if (c == EBLC_OK) c = cuda_status(cudaStreamSynchronize(st), "d2h sync");
     return c;
 }
@@ -609,18 +618,18 @@ EBLC_API eblc_status_t eblc_decompress(eblc_plan_t p, const eblc_execution_t *ex
     st = p->host_stream;
     da.in = p->stage_out;
     da.out = p->stage_in;
+    timing_begin(p, st);  // the "call" pair spans the stream copy in through the output copy back
     if ((s = cuda_status(cudaMemcpyAsync(p->stage_out, d_in, info.total, cudaMemcpyHostToDevice, st), "h2d")) !=
         EBLC_OK)
         return s;
-    timing_begin(p, st);
     timing_mark(p, st, true, "decode");
     s = cuda_status(launch_decode(da, p->num_sms, st), "decode launch");
     timing_mark(p, st, false, nullptr);
-    timing_end(p, st);
     if (s != EBLC_OK) return s;
     if (p->n && (s = cuda_status(cudaMemcpyAsync(d_out, p->stage_in, 4 * p->n, cudaMemcpyDeviceToHost, st),
                                  "d2h")) != EBLC_OK)
         return s;
+    timing_end(p, st);
     if ((s = cuda_status(cudaMemcpyAsync(p->h_err, p->dec_err, 4, cudaMemcpyDeviceToHost, st), "err")) != EBLC_OK ||
         (s = cuda_status(cudaMemsetAsync(p->dec_err, 0, 4, st), "err clear")) != EBLC_OK ||
         (s = cuda_status(cudaStreamSynchronize(st), "decompress sync")) != EBLC_OK)

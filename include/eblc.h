@@ -125,7 +125,9 @@ typedef struct {
 /* Device timing of the last call, recorded when the plan was created with
  * the option "timing=1": CUDA events on the call's stream around each kernel
  * launch, plus one entry "call" from the first launch to the end of the
- * call's last device operation (for compress: the result readback).        */
+ * call's last device operation (for compress: the result readback).  For
+ * the HOST execution kind "call" spans the host-to-device copy of the input
+ * through the device-to-host copy of the output.                           */
 typedef struct {
     char name[24];      /* "range", "encode", "decode", "call"          */
     float ms;           /* elapsed device time                          */

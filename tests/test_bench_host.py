@@ -1,0 +1,105 @@
+"""Host logic of the benchmark, on CPU: the cross-rank reductions that turn
+per-rank timings into the job's numbers (world size 2 over gloo, the same
+calls the multi-GPU run makes over NCCL), the JSON line contract, and the
+reference arm's rank handling."""
+import io
+import json
+import os
+import socket
+import sys
+from contextlib import redirect_stdout
+
+import numpy as np
+import pytest
+
+import bench
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # ranks time different amounts; the job time is the slowest rank's
+        t = bench.max_over_ranks([1.0 + rank, 5.0 - rank, 0.25 * rank], world)
+        # every rank processed its own replica: bytes add up
+        b = bench.sum_over_ranks([4.0 * (1 << 20) * (rank + 1)], world)
+        q.put((rank, t, b))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_rank_reductions_gloo_world2():
+    import torch.multiprocessing as mp
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, t, b in res:
+        assert t == [2.0, 5.0, 0.25]
+        assert b == [4.0 * (1 << 20) * 3]
+
+
+def test_single_rank_reductions_are_identity():
+    assert bench.max_over_ranks([3.0, 1.0], 1) == [3.0, 1.0]
+    assert bench.sum_over_ranks([2.5], 1) == [2.5]
+
+
+class _Args:
+    steps = 4
+    warmup = 3
+    workload = "field512cube_spikes"
+    elements = None
+    no_cpu_baseline = True
+
+
+def test_report_line_contract(monkeypatch):
+    """One JSON line with every key the benchmark contract names; value is the
+    whole job's input bytes over the slowest rank's compress + decompress time."""
+    n, nbytes, world = 1 << 20, 600_000, 2
+    t_comp, t_dec = 0.004, 0.002
+    kern = {"range": [0.1] * 4, "encode": [0.6] * 4, "decode": [0.5] * 4}
+    e2e = {"value": 12.0, "unit": "GB/s", "h2d_bytes_per_step": 4 * n + nbytes, "d2h_bytes_per_step": nbytes + 4 * n}
+    clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 3}
+    total = 4.0 * n * _Args.steps * world
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.report(_Args, world, n, nbytes, t_comp, t_dec, t_comp, t_dec, total, (t_comp + t_dec) / _Args.steps,
+                     kern, e2e, 3, clk, np.zeros(n, np.float32), 64, "rel", 1e-3)
+    lines = [ln for ln in buf.getvalue().splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+              "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
+        assert k in d, k
+    assert d["n_gpus"] == world and d["scaling"] == "weak" and d["higher_is_better"] is True
+    assert d["value"] == pytest.approx(total / (t_comp + t_dec) / 1e9, rel=1e-3)
+    assert d["config"]["workload"] == "field512cube_spikes"
+    r = d["roofline"]
+    assert r["bound"] == "hbm" and r["kernel"] == "encode" and r["unit"] == "GB/s"
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"], abs=1e-4)
+    assert d["gpu_launches"] == 3 * _Args.steps
+    assert d["ratio"] == pytest.approx(4.0 * n / nbytes, rel=1e-4)
+
+
+def test_reference_arm_other_ranks_exit_quietly(monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        assert bench.run_reference(_Args) == 0
+    assert buf.getvalue() == ""
