@@ -293,9 +293,9 @@ cudaError_t launch_t(const DecodeArgs &a, int num_sms, cudaStream_t stream) {
 
 cudaError_t launch_decode(const DecodeArgs &a, int num_sms, cudaStream_t stream) {
     switch (a.block) {
-        case 32: return launch_t<4, 8>(a, num_sms, stream);
-        case 64: return launch_t<4, 16>(a, num_sms, stream);
-        case 128: return launch_t<4, 32>(a, num_sms, stream);
+        case 32: return launch_t<8, 4>(a, num_sms, stream);
+        case 64: return launch_t<8, 8>(a, num_sms, stream);
+        case 128: return launch_t<8, 16>(a, num_sms, stream);
         case 256: return launch_t<8, 32>(a, num_sms, stream);
         default: return cudaErrorInvalidValue;
     }

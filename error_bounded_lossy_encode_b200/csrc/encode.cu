@@ -67,6 +67,7 @@ struct __align__(128) EncSmem {
     uint32_t agg_count[kD];               // compute warps that have added to agg
     int32_t tile_id[kS];
     uint64_t full[kS], empty[kS], computed[kD];
+    uint64_t written[kD];                 // completes once per use of the slot: its tile is written out
     Bound bound;
 };
 
@@ -248,7 +249,6 @@ __device__ void compute_warp(EncSmem &sm, const EncodeArgs &a, int cw, int ln) {
     uint32_t oldest = 0;  // oldest CTA iteration whose packed words still occupy this warp's ring
     uint32_t head = 0;    // ring offset after the newest tile's words
     uint32_t i = 0;
-    uint64_t t0 = 0;
     for (;; ++i) {
         // Reclaim ring space of tiles already written out, then find room for a
         // worst-case tile: a free slot and kWarpMax contiguous ring words.
@@ -269,14 +269,9 @@ __device__ void compute_warp(EncSmem &sm, const EncodeArgs &a, int cw, int ln) {
                     break;
                 }
             }
-            if (t0 == 0) t0 = globaltimer_ns();
-            if (globaltimer_ns() - t0 > a.wait_ns) {
-                if (ln == 0) atomicOr(a.err, kErrTimeout);
-                return;
-            }
-            __nanosleep(64);
+            // No room: sleep on the oldest pending tile's write-out (oldest < i here).
+            if (!mbar_wait(&sm.written[oldest % kD], (oldest / kD) & 1, a.wait_ns, a.err)) return;
         }
-        t0 = 0;
         const int s = i % kS, q = i % kD;
         if (!mbar_wait(&sm.full[s], (i / kS) & 1, a.wait_ns, a.err)) return;
         const int tile = sm.tile_id[s];
@@ -313,15 +308,9 @@ __device__ void compute_warp(EncSmem &sm, const EncodeArgs &a, int cw, int ln) {
     // Tell both look-back warps that this CTA has no more tiles: iterations i
     // and i + 1 get tile -1.  Their slots must be free of pending tiles first.
     while (i - oldest > (uint32_t)(kD - kLookbackWarps)) {
-        if (!slot_done(sm, oldest)) {
-            if (t0 == 0) t0 = globaltimer_ns();
-            if (globaltimer_ns() - t0 > a.wait_ns) {
-                if (ln == 0) atomicOr(a.err, kErrTimeout);
-                return;
-            }
-            __nanosleep(64);
-            continue;
-        }
+        if (!slot_done(sm, oldest) &&
+            !mbar_wait(&sm.written[oldest % kD], (oldest / kD) & 1, a.wait_ns, a.err))
+            return;
         ++oldest;
     }
     if (ln == 0) {
@@ -574,6 +563,7 @@ __device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
         if (ln == 0) {
             __threadfence_block();
             *reinterpret_cast<volatile uint32_t *>(&sm.done[q]) = i + 1;
+            mbar_arrive(&sm.written[q]);
         }
     }
 }
@@ -624,6 +614,7 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const EncodeArgs a)
         }
         for (int q = 0; q < kD; ++q) {
             mbar_init(&sm.computed[q], kNW);
+            mbar_init(&sm.written[q], 1);
             sm.done[q] = 0u;
             sm.agg[q] = 0ull;
             sm.agg_count[q] = 0u;

@@ -5,8 +5,9 @@
 // relative bound eb = rel * (max - min) must be known before any code is
 // produced.  This is the compulsory first read of the input in relative mode.
 //
-// HBM-bound: 4 bytes read per element, no writes.  Persistent grid of
-// 8 CTAs x 256 threads per SM; each thread keeps 4 float4 loads in flight.
+// HBM-bound: 4 bytes read per element, no writes.  Persistent grid of one
+// wave of 256-thread CTAs; each thread keeps 8 float4 loads in flight
+// (fetched with a 256-byte L2 prefetch hint).
 // The array is walked from its end to its start so the lowest addresses are
 // the last read and are still in L2 when the encoder starts at tile 0.
 #include "common.cuh"
@@ -16,12 +17,21 @@ namespace eblc {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = 8;
 
 __device__ __forceinline__ void fold(float v, float &lo, float &hi) {
-    const bool finite = fabsf(v) < __int_as_float(0x7f800000);  // false for NaN and +-Inf
-    lo = fminf(lo, finite ? v : __int_as_float(0x7f800000));
-    hi = fmaxf(hi, finite ? v : __int_as_float(0xff800000));
+    // +-Inf become NaN, which fminf / fmaxf ignore (as they ignore NaN itself)
+    const float f = (fabsf(v) < __int_as_float(0x7f800000)) ? v : __int_as_float(0x7fffffff);
+    lo = fminf(lo, f);
+    hi = fmaxf(hi, f);
+}
+
+__device__ __forceinline__ float4 ld_nc_256(const float4 *p) {
+    float4 v;
+    asm volatile("ld.global.nc.L2::256B.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
 }
 
 __global__ void __launch_bounds__(kThreads) range_kernel(RangeArgs a) {
@@ -36,7 +46,7 @@ __global__ void __launch_bounds__(kThreads) range_kernel(RangeArgs a) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const uint64_t i = base + u * stride + tid;
-            v[u] = (i < n4) ? __ldg(in4 + (n4 - 1 - i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[u] = (i < n4) ? ld_nc_256(in4 + (n4 - 1 - i)) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
@@ -108,7 +118,15 @@ __global__ void __launch_bounds__(kThreads) range_kernel(RangeArgs a) {
 
 }  // namespace
 
-int range_grid(int num_sms) { return num_sms * 8; }
+// One wave of resident CTAs (occupancy is set by the registers of the
+// 8-deep load unroll), at most 8 per SM.
+int range_grid(int num_sms) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, range_kernel, kThreads, 0) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    return num_sms * (per_sm < 8 ? per_sm : 8);
+}
 
 cudaError_t launch_range(const RangeArgs &a, int grid, cudaStream_t stream) {
     range_kernel<<<grid, kThreads, 0, stream>>>(a);
