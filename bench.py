@@ -141,16 +141,21 @@ class ClockSampler:
 # ----------------------------------------------------------------------------------------------
 # workload
 
-def workload(name: str, elements: int | None = None):
+def workload(name: str, elements: int | None = None, rel=None, abs_=None, block=None):
+    """The named standard workload and its options; rel / abs_ / block override them."""
     from error_bounded_lossy_encode_b200 import workloads as WL
 
     x = WL.standard(name)
     if elements:
         x = np.ascontiguousarray(x[:elements])
     o = WL.options_of(name)
-    block = o.pop("block")
+    blk = o.pop("block")
     mode, bound = next(iter(o.items()))
-    return x, block, mode, bound
+    if rel is not None:
+        mode, bound = "rel", rel
+    if abs_ is not None:
+        mode, bound = "abs", abs_
+    return x, (block or blk), mode, bound
 
 
 def options_string(block, mode, bound, timing=False):
@@ -218,7 +223,7 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
-    x, block, mode, bound = workload(args.workload, args.elements)
+    x, block, mode, bound = workload(args.workload, args.elements, args.rel, args.abs, args.block)
     for _ in range(args.warmup):
         cpu_oracle_sample(x, block, mode, bound)
     t0 = time.perf_counter()
@@ -256,7 +261,7 @@ def run_ours(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    x_np, block, mode, bound = workload(args.workload, args.elements)
+    x_np, block, mode, bound = workload(args.workload, args.elements, args.rel, args.abs, args.block)
     n = x_np.size
     st, plan = E.eblc_plan_create([n], None, options_string(block, mode, bound, timing=True))
     if st != E.EBLC_OK:
@@ -443,6 +448,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--elements", type=int, default=None, help="use only the first N elements of the workload")
+    ap.add_argument("--rel", type=float, default=None, help="override the workload's bound: relative")
+    ap.add_argument("--abs", type=float, default=None, help="override the workload's bound: absolute")
+    ap.add_argument("--block", type=int, default=None, choices=(32, 64, 128, 256), help="override the block size")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)

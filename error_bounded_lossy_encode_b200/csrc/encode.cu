@@ -260,11 +260,14 @@ __device__ void compute_warp(EncSmem &sm, const EncodeArgs &a, int cw, int ln) {
                     start = 0;
                     break;
                 }
+                // Pending words occupy [tail, head), wrapped when head < tail.  A
+                // slice never ends exactly at tail, so head == tail means that no
+                // pending word is in the ring.
                 const uint32_t tail = sm.ringpos[oldest % kD][cw];
                 if (head >= tail) {
                     if (head + kWarpMax <= kRing) { start = head; break; }
-                    if (kWarpMax <= tail) { start = 0; break; }
-                } else if (head + kWarpMax <= tail) {
+                    if (kWarpMax < tail) { start = 0; break; }
+                } else if (head + kWarpMax < tail) {
                     start = head;
                     break;
                 }

@@ -65,6 +65,9 @@ class _Args:
     workload = "field512cube_spikes"
     elements = None
     no_cpu_baseline = True
+    rel = None
+    abs = None
+    block = None
 
 
 def test_report_line_contract(monkeypatch):

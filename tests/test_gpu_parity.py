@@ -182,3 +182,16 @@ def test_parity_many_tiles_per_cta(torch_cuda, orc, block):
     x[rng.random(n) < 1e-3] *= 1e3
     _run_parity(orc, x, block, rel=1e-3)
     _run_parity(orc, x, block, abs=1e-4)
+
+
+@pytest.mark.parametrize("block", (32, 256))
+def test_parity_full_width_slices(torch_cuda, orc, block):
+    """Every block at width 32 (codes alternate between +-(2^30 - 64), abs
+    bound 0.5, so x' = x and there are no outliers): each compute warp's
+    part of a tile is the largest it can be, and several tiles per CTA
+    cycle its packed-word buffer through every wrap-around position."""
+    n = 4096 * 148 * 2 * 6 + 4096 - 3
+    x = np.where(np.arange(n) % 2 == 0, 1.0, -1.0) * float(2 ** 30 - 64)
+    want = _run_parity(orc, x.astype(np.float32), block, abs=0.5)
+    h = SC.header(want)
+    assert h["m"] == 0 and h["W"] == n  # 32-bit codes: one word per element
