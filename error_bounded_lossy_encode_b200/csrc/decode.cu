@@ -9,7 +9,7 @@
 // The chunk index gives every chunk's record offset, so chunks decode
 // independently: no scan, no inter-CTA communication, no scratch memory.
 //
-// CTA organisation (288 threads, 2 CTAs per SM, persistent grid, chunk
+// CTA organisation (288 threads, 3 CTAs per SM, persistent grid, chunk
 // t handled by CTA t mod grid):
 //   warps 0..7  compute: warp-tiles of 32*V elements (V consecutive
 //               elements per lane; a block of B elements spans B/V lanes).
@@ -18,7 +18,7 @@
 //               is a lane-serial sum plus a segmented warp scan.
 //   warp 8      producer: reads the chunk index and streams each record
 //               (payload, and the outlier list when it fits) and the
-//               chunk's width bytes into a 3-stage shared-memory ring with
+//               chunk's width bytes into a 2-stage shared-memory ring with
 //               bulk async copies completing on mbarriers.
 // Chunks without outliers store straight from registers (128-bit
 // coalesced stores); chunks with outliers go through a shared-memory tile
@@ -30,7 +30,7 @@ namespace eblc {
 namespace {
 
 constexpr int kNW = 8;
-constexpr int kS = 3;
+constexpr int kS = 2;
 constexpr int kThreads = (kNW + 1) * 32;
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kStagedOutliers = 1024;                 // outliers staged with the payload
@@ -257,7 +257,7 @@ __device__ void producer_warp(DecSmem &sm, const DecodeArgs &a, int ln) {
 }
 
 template <int V, int LPB>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     DecSmem &sm = *reinterpret_cast<DecSmem *>(smem_raw);
     const int warp = threadIdx.x / 32, ln = threadIdx.x % 32;
@@ -283,7 +283,7 @@ cudaError_t launch_t(const DecodeArgs &a, int num_sms, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const uint64_t nc = (a.n + kChunk - 1) / kChunk;
     if (nc == 0) return cudaSuccess;
-    const uint64_t want = (uint64_t)num_sms * 2;
+    const uint64_t want = (uint64_t)num_sms * 3;
     const int grid = (int)(want < nc ? want : nc);
     decode_kernel<V, LPB><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();

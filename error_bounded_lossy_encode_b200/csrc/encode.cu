@@ -13,7 +13,7 @@
 //   (launchGenericChunkFusion: scan/pack tail) -- here a single-pass
 //   decoupled look-back instead of a separate scan and gather.
 //
-// CTA organisation (352 threads, 2 CTAs per SM, cooperative persistent grid;
+// CTA organisation (384 threads, 2 CTAs per SM, cooperative persistent grid;
 // tile t = chunk t of 4096 elements is processed by CTA t mod gridDim.x):
 //   warps 0..7   compute: each owns a contiguous 512-element slice of the
 //                tile, held as warp-tiles of 32*V elements (V = 8 consecutive
@@ -26,12 +26,14 @@
 //                to their final position once the tile's prefix is known,
 //                up to kD - 1 tiles later, so look-back latency overlaps with
 //                the compute of later tiles.
-//   warps 8, 9   look-back (CTA tile iterations i with i mod 2 = warp - 8):
-//                resolve the exclusive prefix of a tile from the
-//                predecessors' status words (320 per coalesced L2 round trip), publish
-//                its inclusive prefix, write the chunk index entry (and the
-//                header for the last tile).
-//   warp 10      producer: streams the CTA's tiles into a 3-stage shared-
+//   warps 8..10  look-back and write-out (CTA tile iterations i with
+//                i mod 3 = warp - 8): resolve the exclusive prefix of a tile
+//                from the predecessors' status words (320 per coalesced L2
+//                round trip), publish its inclusive prefix, write the chunk
+//                index entry (and the header for the last tile), then copy
+//                the compute warps' packed words, the outliers and the width
+//                bytes to their final positions.
+//   warp 11      producer: streams the CTA's tiles into a 3-stage shared-
 //                memory ring with bulk async copies (cp.async.bulk,
 //                completion on mbarriers).
 // Every wait is bounded (kErrTimeout); every global store is checked against
@@ -45,7 +47,7 @@ namespace {
 constexpr int kNW = 8;                    // compute warps
 constexpr int kS = 3;                     // input stages
 constexpr int kD = 8;                     // tile slots: at most kD - 1 tiles computed but not finished
-constexpr int kLookbackWarps = 2;
+constexpr int kLookbackWarps = 3;
 constexpr int kProducerWarp = kNW + kLookbackWarps;
 constexpr int kThreads = (kNW + kLookbackWarps + 1) * 32;
 constexpr int kWindow = 10;               // look-back rows of 32 status words per round trip
@@ -308,8 +310,9 @@ __device__ void compute_warp(EncSmem &sm, const EncodeArgs &a, int cw, int ln) {
         }
         head = start + words;
     }
-    // Tell both look-back warps that this CTA has no more tiles: iterations i
-    // and i + 1 get tile -1.  Their slots must be free of pending tiles first.
+    // Tell the look-back warps that this CTA has no more tiles: iterations
+    // i .. i + kLookbackWarps - 1 get tile -1.  Their slots must be free of
+    // pending tiles first.
     while (i - oldest > (uint32_t)(kD - kLookbackWarps)) {
         if (!slot_done(sm, oldest) &&
             !mbar_wait(&sm.written[oldest % kD], (oldest / kD) & 1, a.wait_ns, a.err))
