@@ -346,18 +346,17 @@ __device__ __forceinline__ void write_tile(EncSmem &sm, const EncodeArgs &a, con
     const float *xin = a.in + (uint64_t)tile * kChunk;
 #pragma unroll 1
     for (int c = 0; c < kNW; ++c) {
-        const uint32_t words = sm.totals[q][c][0], pos = sm.ringpos[q][c];
+        const uint32_t words = sm.totals[q][c][0], pos = sm.ringpos[q][c], mc = sm.totals[q][c][1];
         const uint64_t w0 = (uint64_t)rec + __shfl_sync(kFull, wpw, c);
         const uint32_t *src = sm.ring[c] + pos;
-        for (uint32_t j = ln; j < words; j += 32) {
-            if (w0 + j < cap_words)
-                st_cs_u32(recs + w0 + j, src[j]);
-            else
-                over = true;
-        }
-        const uint32_t omask = sm.omask[q][c][ln];
+        uint32_t *dst = recs + w0;
+        // words that fit in the caller's capacity (all of them unless it is too small)
+        const uint32_t lim = (w0 >= cap_words) ? 0u : (uint32_t)min((uint64_t)words, cap_words - w0);
+        over |= lim < words;
+        for (uint32_t j = ln; j < lim; j += 32) st_cs_u32(dst + j, src[j]);
         const uint32_t obase = __shfl_sync(kFull, wpo, c);
-        if (__any_sync(kFull, omask != 0u)) {
+        if (mc != 0u) {
+            const uint32_t omask = sm.omask[q][c][ln];
             uint32_t ord_base = 0;
 #pragma unroll 1
             for (int k = 0; k < kWPW; ++k) {
@@ -395,12 +394,10 @@ __device__ __forceinline__ void write_tile(EncSmem &sm, const EncodeArgs &a, con
         const uint32_t nwords = (uint32_t)((bend - b0) / 4);
         const uint32_t *ws = reinterpret_cast<const uint32_t *>(sm.width[q]);
         uint32_t *wd = reinterpret_cast<uint32_t *>(a.out + L.width_off + b0);
-        for (uint32_t j = ln; j < nwords; j += 32) {
-            if (L.width_off + b0 + 4 * j + 4 <= a.out_cap)
-                wd[j] = ws[j];
-            else
-                over = true;
-        }
+        const uint64_t room = (a.out_cap > L.width_off + b0) ? (a.out_cap - L.width_off - b0) / 4 : 0;
+        const uint32_t nw = (uint32_t)min((uint64_t)nwords, room);
+        over |= nw < nwords;
+        for (uint32_t j = ln; j < nw; j += 32) wd[j] = ws[j];
     }
     if (__any_sync(kFull, over) && ln == 0) atomicOr(a.err, kErrCapacity);
 }
@@ -629,10 +626,7 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const EncodeArgs a)
         const float vmin = a.abs_mode ? 0.0f : a.range[0];
         const float vmax = a.abs_mode ? 0.0f : a.range[1];
         sm.bound = resolve_bound(a.abs_mode, a.bound, vmin, vmax);
-        if (blockIdx.x == 0) {
-            *a.counter_next = 0u;
-            *a.err_next = 0u;
-        }
+        if (blockIdx.x == 0) *a.err_next = 0u;
     }
     __syncthreads();
 

@@ -33,8 +33,6 @@ struct EncodeArgs {
     const float *range;       // vmin, vmax from the range kernel (relative mode)
     uint64_t *status;         // this call's look-back words [ntiles], zero on entry
     uint64_t *status_next;    // the other call parity's words, cleared here
-    uint32_t *counter;        // this call's tile counter, zero on entry
-    uint32_t *counter_next;   // cleared here
     uint32_t *err;            // this call's error word
     uint32_t *err_next;       // cleared here
     uint64_t *result;         // [W, m, total, R] written by the last tile

@@ -7,7 +7,7 @@
 // forbidden or would synchronise the device, and callers that must not grow
 // the device footprint behind their back.  They can still compress with this
 // entry point: it needs no plan, and the scratch the range and encode kernels
-// use (look-back status words, tile counters, error words, range partials,
+// use (look-back status words, error words, range partials,
 // the result block) lives in one file-scope __device__ array of fixed size,
 // which every GPU that loads this library holds until the process exits.
 // The caller passes the input and the output buffer, as with eblc_compress.
@@ -29,10 +29,9 @@ constexpr int kMaxDevices = 64;
 
 struct NoallocScratch {
     // cleared at the start of every call
-    uint32_t counter[2];
     uint32_t err[2];
     uint32_t range_counter;
-    uint32_t pad[3];
+    uint32_t pad[5];
     uint64_t result[8];
     // written before being read within a call
     float range[4];
@@ -110,8 +109,6 @@ extern "C" EBLC_API eblc_status_t eblc_compress_noalloc(const float *d_in, uint6
     ea.range = S->range;
     ea.status = S->status[0];
     ea.status_next = S->status[1];
-    ea.counter = &S->counter[0];
-    ea.counter_next = &S->counter[1];
     ea.err = &S->err[0];
     ea.err_next = &S->err[1];
     ea.result = S->result;

@@ -51,8 +51,8 @@ bool log_enabled() {
         }                                          \
     } while (0)
 
-// Device scratch owned by a plan: look-back status words and tile counters
-// for both call parities, error words, range partials, readback block.
+// Device scratch owned by a plan: look-back status words for both call
+// parities, error words, range partials, readback block.
 struct Readback {
     uint64_t result[8];  // W, m, total, R, eb bits, step|inv2eb, vmin|vmax, unused
     uint32_t err[2];
@@ -85,7 +85,6 @@ struct eblc_plan_s {
 
     void *scratch = nullptr;
     uint64_t *status[2] = {};
-    uint32_t *counter[2] = {};
     Readback *d_rb = nullptr;       // device copy of the readback block
     uint32_t *dec_err = nullptr;
     float2 *partials = nullptr;
@@ -295,8 +294,6 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
     ea.range = p->range;
     ea.status = p->status[par];
     ea.status_next = p->status[par ^ 1];
-    ea.counter = p->counter[par];
-    ea.counter_next = p->counter[par ^ 1];
     ea.err = &p->d_rb->err[par];
     ea.err_next = &p->d_rb->err[par ^ 1];
     ea.result = p->d_rb->result;
@@ -471,8 +468,6 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
         off = 0;
         p->status[0] = carve<uint64_t>(base, &off, ntiles);
         p->status[1] = carve<uint64_t>(base, &off, ntiles);
-        p->counter[0] = carve<uint32_t>(base, &off, 1);
-        p->counter[1] = carve<uint32_t>(base, &off, 1);
         p->d_rb = carve<Readback>(base, &off, 1);
         p->dec_err = carve<uint32_t>(base, &off, 1);
         p->partials = carve<float2>(base, &off, p->range_grid);
