@@ -10,6 +10,7 @@ Functions keep the C names::
     st, plan = eblc_plan_create(dims, strides=None, options="rel=1e-3,block=64")
     st, lim  = eblc_plan_get_limits(plan)
     st, nbytes = eblc_compress(plan, cuda_exec(stream), d_in, d_out, capacity, sidecar)
+    st = eblc_compress_async(plan, cuda_exec(stream), d_in, d_out, capacity, d_result)   # no host sync
     st = eblc_decompress(plan, cuda_exec(stream), d_stream, nbytes, sidecar, d_out)
     st = eblc_check(plan, cuda_exec(stream))
     eblc_plan_destroy(plan)
@@ -52,11 +53,17 @@ class eblc_sidecar_t(ctypes.Structure):
                 ("inv2eb", ctypes.c_float)]
 
 
+class eblc_async_result_t(ctypes.Structure):
+    _fields_ = [("compressed_bytes", ctypes.c_uint64), ("payload_words", ctypes.c_uint64),
+                ("n_outliers", ctypes.c_uint64), ("status", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
+
+
 class eblc_kernel_time_t(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 24), ("ms", ctypes.c_float), ("launches", ctypes.c_uint32)]
 
 
 assert ctypes.sizeof(eblc_sidecar_t) == 64
+assert ctypes.sizeof(eblc_async_result_t) == 32
 
 
 def _fields(s: ctypes.Structure) -> dict:
@@ -87,6 +94,8 @@ def lib() -> ctypes.CDLL:
     L.eblc_compress.argtypes = [P, ctypes.POINTER(eblc_execution_t), P, P, ctypes.c_size_t,
                                 ctypes.POINTER(ctypes.c_size_t), P]
     L.eblc_compress.restype = i32
+    L.eblc_compress_async.argtypes = [P, ctypes.POINTER(eblc_execution_t), P, P, ctypes.c_size_t, P]
+    L.eblc_compress_async.restype = i32
     L.eblc_decompress.argtypes = [P, ctypes.POINTER(eblc_execution_t), P, ctypes.c_size_t, P, P]
     L.eblc_decompress.restype = i32
     L.eblc_check.argtypes = [P, ctypes.POINTER(eblc_execution_t)]
@@ -141,6 +150,20 @@ def eblc_compress(plan, exec_: eblc_execution_t, d_in: int, d_out: int, out_capa
                              ctypes.c_void_p(d_out or None), out_capacity, ctypes.byref(nbytes),
                              None if sidecar is None else ctypes.byref(sidecar))
     return st, int(nbytes.value)
+
+
+def eblc_compress_async(plan, exec_: eblc_execution_t, d_in: int, d_out: int, out_capacity: int,
+                        d_result: int) -> int:
+    """Queue a compress on exec_'s stream; the device writes an
+    eblc_async_result_t (32 bytes) at d_result.  Returns the queueing status."""
+    return lib().eblc_compress_async(plan, ctypes.byref(exec_), ctypes.c_void_p(d_in or None),
+                                     ctypes.c_void_p(d_out or None), out_capacity, ctypes.c_void_p(d_result or None))
+
+
+def async_result(raw) -> dict:
+    """Decode the 32 bytes of an eblc_async_result_t (e.g. a uint8 tensor copied to the host)."""
+    r = eblc_async_result_t.from_buffer_copy(bytes(raw))
+    return _fields(r)
 
 
 def eblc_decompress(plan, exec_: eblc_execution_t, d_in: int, compressed_bytes: int, sidecar, d_out: int) -> int:

@@ -40,6 +40,7 @@
 // the caller's capacity (kErrCapacity).
 #include "common.cuh"
 #include "kernels.h"
+#include "../../include/eblc.h"
 
 namespace eblc {
 namespace {
@@ -69,6 +70,7 @@ struct __align__(128) EncSmem {
     uint32_t agg_count[kD];               // compute warps that have added to agg
     int32_t tile_id[kS];
     uint64_t full[kS], empty[kS], computed[kD];
+    uint64_t *st_cur, *st_next;           // this call's look-back words, the other array
     uint64_t written[kD];                 // completes once per use of the slot: its tile is written out
     Bound bound;
 };
@@ -304,7 +306,7 @@ __device__ void compute_warp(EncSmem &sm, const EncodeArgs &a, int cw, int ln) {
                 sm.agg_count[q] = 0;
                 const uint32_t PW = (uint32_t)t, MT = (uint32_t)(t >> 32);
                 if (tile != a.stall_tile)
-                    st_relaxed_gpu(&a.status[tile], pack_status(PW + 2u * MT, MT, tile == 0));
+                    st_relaxed_gpu(&sm.st_cur[tile], pack_status(PW + 2u * MT, MT, tile == 0));
             }
             mbar_arrive(&sm.computed[q]);
         }
@@ -461,8 +463,8 @@ __device__ void write_header(const EncodeArgs &a, const Layout &L, const Bound &
 // aggregate: polls the nearest missing one with back-off (bounded by
 // wait_ns, and given up at once when another wait of the launch has timed
 // out), then reads the window again.
-__device__ __forceinline__ void look_back(const EncodeArgs &a, int tile, int stop, uint64_t known, int ln,
-                                          uint32_t &exR, uint32_t &exM) {
+__device__ __forceinline__ void look_back(const EncodeArgs &a, const uint64_t *status, int tile, int stop,
+                                          uint64_t known, int ln, uint32_t &exR, uint32_t &exM) {
     exR = 0;
     exM = 0;
     int base = tile - 1;  // nearest predecessor not yet summed
@@ -473,7 +475,7 @@ __device__ __forceinline__ void look_back(const EncodeArgs &a, int tile, int sto
 #pragma unroll
         for (int j = 0; j < kWindow; ++j) {
             const int p = base - 32 * j - ln;
-            v[j] = (p > stop) ? ld_relaxed_gpu(&a.status[p]) : (p == stop ? known : pack_status(0, 0, true));
+            v[j] = (p > stop) ? ld_relaxed_gpu(&status[p]) : (p == stop ? known : pack_status(0, 0, true));
         }
         uint32_t sr = 0, sm_ = 0;
         int found = 0, miss_row = -1;
@@ -497,7 +499,7 @@ __device__ __forceinline__ void look_back(const EncodeArgs &a, int tile, int sto
             }
         }
         if (miss_row >= 0) {
-            const uint64_t *w = &a.status[base - 32 * miss_row - (__ffs(miss_lanes) - 1)];
+            const uint64_t *w = &status[base - 32 * miss_row - (__ffs(miss_lanes) - 1)];
             if (t0 == 0) t0 = globaltimer_ns();
             while (ld_relaxed_gpu(w) == 0) {
                 if (globaltimer_ns() - t0 > a.wait_ns ||
@@ -548,11 +550,11 @@ __device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
             // other CTAs have almost always published this tile's predecessors
             // of the same wave, so the look-back rarely has to wait.
             if (!mbar_wait(&sm.computed[(i + 1) % kD], ((i + 1) / kD) & 1, a.wait_ns, a.err)) return;
-            look_back(a, tile, -1, pack_status(0, 0, true), ln, exR, exM);
-            if (ln == 0 && publish) st_relaxed_gpu(&a.status[tile], pack_status(exR + Rt, exM + MT, true));
+            look_back(a, sm.st_cur, tile, -1, pack_status(0, 0, true), ln, exR, exM);
+            if (ln == 0 && publish) st_relaxed_gpu(&sm.st_cur[tile], pack_status(exR + Rt, exM + MT, true));
         }
         if (ln == 0) {
-            a.status_next[tile] = 0ull;
+            sm.st_next[tile] = 0ull;
             const uint64_t io_off = L.index_off + 8ull * (uint64_t)tile;
             if (io_off + 8 <= a.out_cap)
                 *reinterpret_cast<uint64_t *>(a.out + io_off) = (uint64_t)exR | ((uint64_t)exM << 32);
@@ -626,7 +628,9 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const EncodeArgs a)
         const float vmin = a.abs_mode ? 0.0f : a.range[0];
         const float vmax = a.abs_mode ? 0.0f : a.range[1];
         sm.bound = resolve_bound(a.abs_mode, a.bound, vmin, vmax);
-        if (blockIdx.x == 0) *a.err_next = 0u;
+        const uint64_t par = *a.epoch & 1u;
+        sm.st_cur = a.status + par * a.ntiles;
+        sm.st_next = a.status + (par ^ 1u) * a.ntiles;
     }
     __syncthreads();
 
@@ -659,7 +663,29 @@ cudaError_t launch_t(const EncodeArgs &a, int num_sms, cudaStream_t stream) {
                                        dim3(kThreads), params, smem, stream);
 }
 
+__global__ void finish_kernel(const FinishArgs f) {
+    const uint32_t err = *f.err;
+    f.result[7] = err;
+    *f.err = 0u;
+    *f.epoch += 1u;
+    if (f.user) {
+        const uint32_t status = (err & kErrTimeout)    ? (uint32_t)EBLC_TIMEOUT
+                                : (err & kErrCapacity) ? (uint32_t)EBLC_CAPACITY
+                                : (err & kErrCorrupt)  ? (uint32_t)EBLC_CORRUPT
+                                                       : (uint32_t)EBLC_OK;
+        f.user[0] = f.result[2];  // stream bytes
+        f.user[1] = f.result[0];  // payload words
+        f.user[2] = f.result[1];  // outliers
+        f.user[3] = status;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_finish(const FinishArgs &f, cudaStream_t stream) {
+    finish_kernel<<<1, 1, 0, stream>>>(f);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_encode(const EncodeArgs &a, int num_sms, cudaStream_t stream) {
     switch (a.block) {

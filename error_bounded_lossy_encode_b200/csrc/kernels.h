@@ -31,16 +31,29 @@ struct EncodeArgs {
     int abs_mode;
     double bound;             // relative or absolute bound as requested
     const float *range;       // vmin, vmax from the range kernel (relative mode)
-    uint64_t *status;         // this call's look-back words [ntiles], zero on entry
-    uint64_t *status_next;    // the other call parity's words, cleared here
-    uint32_t *err;            // this call's error word
-    uint32_t *err_next;       // cleared here
-    uint64_t *result;         // [W, m, total, R] written by the last tile
+    uint64_t *status;         // look-back words: two arrays of ntiles; the call uses array
+                              // (*epoch & 1), zero on entry, and clears the other one
+    uint64_t ntiles;          // stride between the two arrays
+    const uint32_t *epoch;    // call counter on the device (advanced by the finish kernel)
+    uint32_t *err;            // error word, zero on entry
+    uint64_t *result;         // [W, m, total, R, eb, step|inv2eb, vmin|vmax] written by the last tile
     uint64_t outlier_cap;
     int64_t stall_tile;       // test hook (-1: off)
     uint64_t wait_ns;         // limit of every device-side wait
 };
 cudaError_t launch_encode(const EncodeArgs &a, int num_sms, cudaStream_t stream);
+
+// One thread, after the encoder on the same stream: result[7] = the call's
+// error word, which it then clears; advances the call counter; and, when
+// `user` is set, writes the caller's result record (compressed bytes,
+// payload words, outliers, status code).
+struct FinishArgs {
+    uint64_t *result;         // the encoder's result block (8 words)
+    uint32_t *err;
+    uint32_t *epoch;
+    uint64_t *user;           // NULL, or 4 words: total, W, m, status | reserved << 32
+};
+cudaError_t launch_finish(const FinishArgs &f, cudaStream_t stream);
 
 // Fused decode: widths + chunk records -> reconstruction with the chunk's
 // outliers written back.

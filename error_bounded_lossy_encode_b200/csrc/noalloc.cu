@@ -29,7 +29,8 @@ constexpr int kMaxDevices = 64;
 
 struct NoallocScratch {
     // cleared at the start of every call
-    uint32_t err[2];
+    uint32_t err;
+    uint32_t epoch;          // stays 0: every call uses look-back array 0, cleared here
     uint32_t range_counter;
     uint32_t pad[5];
     uint64_t result[8];
@@ -107,10 +108,10 @@ extern "C" EBLC_API eblc_status_t eblc_compress_noalloc(const float *d_in, uint6
     ea.abs_mode = abs_mode ? 1 : 0;
     ea.bound = bound;
     ea.range = S->range;
-    ea.status = S->status[0];
-    ea.status_next = S->status[1];
-    ea.err = &S->err[0];
-    ea.err_next = &S->err[1];
+    ea.status = &S->status[0][0];
+    ea.ntiles = kMaxTiles;
+    ea.epoch = &S->epoch;
+    ea.err = &S->err;
     ea.result = S->result;
     ea.outlier_cap = n;
     ea.stall_tile = -1;
@@ -122,7 +123,7 @@ extern "C" EBLC_API eblc_status_t eblc_compress_noalloc(const float *d_in, uint6
         uint32_t err;
     } rb;
     if (cudaMemcpyAsync(rb.result, S->result, sizeof(rb.result), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
-        cudaMemcpyAsync(&rb.err, &S->err[0], sizeof(rb.err), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaMemcpyAsync(&rb.err, &S->err, sizeof(rb.err), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess)
         return EBLC_CUDA_ERROR;
     if (compressed_bytes) *compressed_bytes = (size_t)rb.result[2];

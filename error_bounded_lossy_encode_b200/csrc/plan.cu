@@ -51,11 +51,13 @@ bool log_enabled() {
         }                                          \
     } while (0)
 
-// Device scratch owned by a plan: look-back status words for both call
-// parities, error words, range partials, readback block.
+// Device scratch owned by a plan: look-back status words (two arrays, used
+// alternately by consecutive calls as the device-side call counter says),
+// error word, range partials, readback block.
 struct Readback {
-    uint64_t result[8];  // W, m, total, R, eb bits, step|inv2eb, vmin|vmax, unused
-    uint32_t err[2];
+    uint64_t result[8];  // W, m, total, R, eb bits, step|inv2eb, vmin|vmax, the call's error bits
+    uint32_t err;        // error word of the running call (cleared by the finish kernel)
+    uint32_t epoch;      // calls finished on the device: selects the look-back array
 };
 
 // Per-call device timing (option timing=1): a start/end event pair around
@@ -84,14 +86,14 @@ struct eblc_plan_s {
     uint64_t max_bytes = 0;
 
     void *scratch = nullptr;
-    uint64_t *status[2] = {};
+    uint64_t *status = nullptr;     // 2 x ntiles look-back words
+    uint64_t ntiles = 0;
     Readback *d_rb = nullptr;       // device copy of the readback block
     uint32_t *dec_err = nullptr;
     float2 *partials = nullptr;
     uint32_t *range_counter = nullptr;
     float *range = nullptr;
     int range_grid = 0;
-    int parity = 0;
     Readback *h_rb = nullptr;       // pinned
     uint32_t *h_err = nullptr;      // pinned
 
@@ -269,13 +271,14 @@ eblc_status_t ensure_host_staging(eblc_plan_s *p) {
 // Queue the compress kernels on `st` (device pointers).
 // call_events: record the "call" timing pair around this enqueue (false when
 // the caller brackets a larger span, e.g. the HOST kind's copies).
+// d_user: NULL for the synchronous calls (the result block is copied to the
+// pinned readback), else the caller's device result record (no copy back).
 eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_in, uint8_t *d_out, uint64_t cap,
-                               bool call_events = true) {
+                               bool call_events = true, uint64_t *d_user = nullptr) {
     if (call_events)
         timing_begin(p, st);
     else
         p->timing.count = 0;
-    const int par = p->parity;
     if (!p->abs_mode && p->n > 0) {
         RangeArgs ra{d_in, p->n, p->partials, p->range_counter, p->range};
         timing_mark(p, st, true, "range");
@@ -292,10 +295,10 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
     ea.abs_mode = p->abs_mode;
     ea.bound = p->bound;
     ea.range = p->range;
-    ea.status = p->status[par];
-    ea.status_next = p->status[par ^ 1];
-    ea.err = &p->d_rb->err[par];
-    ea.err_next = &p->d_rb->err[par ^ 1];
+    ea.status = p->status;
+    ea.ntiles = p->ntiles;
+    ea.epoch = &p->d_rb->epoch;
+    ea.err = &p->d_rb->err;
     ea.result = p->d_rb->result;
     ea.outlier_cap = p->outlier_cap;
     ea.stall_tile = p->stall_tile;
@@ -304,16 +307,17 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
     eblc_status_t s = cuda_status(launch_encode(ea, p->num_sms, st), "encode launch");
     timing_mark(p, st, false, nullptr);
     if (s != EBLC_OK) return s;
-    s = cuda_status(cudaMemcpyAsync(p->h_rb, p->d_rb, sizeof(Readback), cudaMemcpyDeviceToHost, st), "readback");
+    FinishArgs fa{p->d_rb->result, &p->d_rb->err, &p->d_rb->epoch, d_user};
+    if ((s = cuda_status(launch_finish(fa, st), "finish launch")) != EBLC_OK) return s;
+    if (!d_user)
+        s = cuda_status(cudaMemcpyAsync(p->h_rb, p->d_rb, sizeof(Readback), cudaMemcpyDeviceToHost, st), "readback");
     if (call_events) timing_end(p, st);
     return s;
 }
 
 eblc_status_t finish_compress(eblc_plan_s *p, size_t *compressed_bytes, void *h_sidecar) {
-    const int par = p->parity;
-    p->parity ^= 1;
     const Readback &rb = *p->h_rb;
-    const uint32_t err = rb.err[par];
+    const uint32_t err = (uint32_t)rb.result[7];
     const uint64_t total = rb.result[2];
     if (compressed_bytes) *compressed_bytes = (size_t)total;
     if (h_sidecar) {
@@ -462,12 +466,12 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
     p->range_grid = range_grid(p->num_sms);
 
     const size_t ntiles = std::max<uint64_t>(p->L.nc, 1);
+    p->ntiles = ntiles;
     size_t off = 0;
     uint8_t *base = nullptr;  // first pass computes the size
     for (int pass = 0; pass < 2; ++pass) {
         off = 0;
-        p->status[0] = carve<uint64_t>(base, &off, ntiles);
-        p->status[1] = carve<uint64_t>(base, &off, ntiles);
+        p->status = carve<uint64_t>(base, &off, 2 * ntiles);
         p->d_rb = carve<Readback>(base, &off, 1);
         p->dec_err = carve<uint32_t>(base, &off, 1);
         p->partials = carve<float2>(base, &off, p->range_grid);
@@ -558,6 +562,31 @@ EBLC_API eblc_status_t eblc_compress(eblc_plan_t p, const eblc_execution_t *exec
     timing_end(p, st);
     if (c == EBLC_OK) c = cuda_status(cudaStreamSynchronize(st), "d2h sync");
     return c;
+}
+
+EBLC_API eblc_status_t eblc_compress_async(eblc_plan_t p, const eblc_execution_t *exec, const float *d_in,
+                                           void *d_out, size_t out_capacity, eblc_async_result_t *d_result) {
+    static_assert(sizeof(eblc_async_result_t) == 32, "async result record is 4 words");
+    if (!p || !exec || !d_result) return EBLC_INVALID_ARG;
+    if (exec->kind == EBLC_EXECUTION_HIP) return EBLC_UNSUPPORTED;
+    if (exec->kind != EBLC_EXECUTION_CUDA) return EBLC_INVALID_ARG;
+    if (!d_out || (p->n && !d_in)) return EBLC_INVALID_ARG;
+    if (!aligned16(d_out) || (d_in && !aligned16(d_in)) || (reinterpret_cast<uintptr_t>(d_result) & 7u))
+        return EBLC_INVALID_ARG;
+    if (out_capacity < p->L.record_off) return EBLC_CAPACITY;
+    DeviceGuard g(p->device);
+    if (!g.ok) return EBLC_CUDA_ERROR;
+    cudaStream_t st = static_cast<cudaStream_t>(exec->stream);
+    // Under stream capture no timing events are recorded (the graph replays
+    // the kernels only).
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return EBLC_CUDA_ERROR;
+    const bool timed = p->timing.on;
+    if (cs != cudaStreamCaptureStatusNone) p->timing.on = false;
+    const eblc_status_t s = enqueue_compress(p, st, d_in, static_cast<uint8_t *>(d_out), out_capacity, true,
+                                             reinterpret_cast<uint64_t *>(d_result));
+    p->timing.on = timed;
+    return s;
 }
 
 EBLC_API eblc_status_t eblc_decompress(eblc_plan_t p, const eblc_execution_t *exec, const void *d_in,

@@ -190,6 +190,42 @@ EBLC_API eblc_status_t eblc_compress(eblc_plan_t plan, const eblc_execution_t *e
                                      void *d_out, size_t out_capacity, size_t *compressed_bytes,
                                      void *h_sidecar);
 
+/* Device-written result of eblc_compress_async (4 words, 8-byte aligned).  */
+typedef struct eblc_async_result_t {
+    uint64_t compressed_bytes;  /* stream length; with EBLC_CAPACITY the length the
+                                   stream needs                                    */
+    uint64_t payload_words;     /* W                                               */
+    uint64_t n_outliers;        /* m                                               */
+    uint32_t status;            /* eblc_status_t of the device work: EBLC_OK,
+                                   EBLC_CAPACITY or EBLC_TIMEOUT                   */
+    uint32_t reserved;
+} eblc_async_result_t;
+
+/*
+ * Compress one snapshot without synchronising the host: every step is
+ * queued on exec->stream (CUDA kind only) and the call returns at once; the
+ * stream length, the counts and the device status are written to *d_result
+ * (device memory, or host memory mapped into the device) by the last queued
+ * kernel.  There is no host synchronisation, memory allocation or host read
+ * inside, so the call may be captured into a CUDA graph and the graph
+ * replayed: the plan keeps its per-call state (which of its two look-back
+ * arrays a call uses) on the device.  Sources: FZGPUModules "Architecture",
+ * MemoryPool (CUDA Graph capture of a pipeline with a preallocated pool);
+ * "DevitoComp provider interface", Provider layout (device work may stay
+ * queued when the call returns).  No sidecar is produced: build one
+ * from the stream header, or pass NULL to eblc_decompress (which then reads
+ * the header, synchronising once).
+ *   d_in, d_out, out_capacity  as for eblc_compress (device pointers)
+ *   d_result   8-byte aligned record, valid once the stream reaches it
+ * Returns EBLC_OK when the work was queued (argument errors and a capacity
+ * below the fixed sections are reported at once); the outcome of the device
+ * work is d_result->status.  Calls on one plan are serialised by the stream
+ * order like every plan call; with timing=1 per-kernel times are recorded
+ * unless the stream is capturing.
+ */
+EBLC_API eblc_status_t eblc_compress_async(eblc_plan_t plan, const eblc_execution_t *exec, const float *d_in,
+                                           void *d_out, size_t out_capacity, eblc_async_result_t *d_result);
+
 /*
  * Decompress one snapshot.
  *   d_in              the stream (compressed_bytes long, 16-byte aligned).

@@ -55,6 +55,7 @@ def test_version_and_status_strings(E):
 def test_struct_sizes(E):
     assert ctypes.sizeof(E.eblc_sidecar_t) == 64
     assert ctypes.sizeof(E.eblc_limits_t) == 72  # matches the static_assert in plan.cu
+    assert ctypes.sizeof(E.eblc_async_result_t) == 32  # matches the static_assert in plan.cu
 
 
 @pytest.mark.parametrize("opts,status", [
