@@ -9,7 +9,7 @@
 // The chunk index gives every chunk's record offset, so chunks decode
 // independently: no scan, no inter-CTA communication, no scratch memory.
 //
-// CTA organisation (288 threads, 3 CTAs per SM, persistent grid, chunk
+// CTA organisation (288 threads, 4 CTAs per SM, persistent grid, chunk
 // t handled by CTA t mod grid):
 //   warps 0..7  compute: warp-tiles of 32*V elements (V consecutive
 //               elements per lane; a block of B elements spans B/V lanes).
@@ -20,9 +20,10 @@
 //               (payload, and the outlier list when it fits) and the
 //               chunk's width bytes into a 2-stage shared-memory ring with
 //               bulk async copies completing on mbarriers.
-// Chunks without outliers store straight from registers (128-bit
-// coalesced stores); chunks with outliers go through a shared-memory tile
-// so the outliers can be written over it before the tile is stored.
+// The reconstruction is stored straight from registers (128-bit coalesced
+// streaming stores); a chunk's outliers are then written over it in global
+// memory, after a barrier of the compute warps orders them behind every
+// reconstruction store of the chunk.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -39,7 +40,6 @@ constexpr uint32_t kRecWords = kChunk + 2 * kStagedOutliers + 4 + 16;  // + alig
 struct __align__(128) DecSmem {
     uint32_t rec[kS][kRecWords];
     uint8_t width[kS][kChunk / 32];
-    float out[kChunk];     // reconstruction of a chunk that has outliers
     uint32_t info[kS][8];  // tile (or -1), valid, PW, mt, adj, staged, rec, corrupt
     uint64_t full[kS], empty[kS];
 };
@@ -123,22 +123,15 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
 #pragma unroll
                 for (int v = 0; v < V; ++v) y[v] = __fmul_rn(__int2float_rn((int32_t)((uint32_t)c[v] + ex)), a.step);
 
-                if (mt == 0) {
-                    if (e0 + V <= valid) {
-#pragma unroll
-                        for (int h = 0; h < V / 4; ++h)
-                            __stcs(reinterpret_cast<float4 *>(gout + e0 + 4 * h),
-                                   make_float4(y[4 * h], y[4 * h + 1], y[4 * h + 2], y[4 * h + 3]));
-                    } else {
-#pragma unroll
-                        for (int v = 0; v < V; ++v)
-                            if (e0 + v < valid) gout[e0 + v] = y[v];
-                    }
-                } else {
+                if (e0 + V <= valid) {
 #pragma unroll
                     for (int h = 0; h < V / 4; ++h)
-                        *reinterpret_cast<float4 *>(&sm.out[e0 + 4 * h]) =
-                            make_float4(y[4 * h], y[4 * h + 1], y[4 * h + 2], y[4 * h + 3]);
+                        __stcs(reinterpret_cast<float4 *>(gout + e0 + 4 * h),
+                               make_float4(y[4 * h], y[4 * h + 1], y[4 * h + 2], y[4 * h + 3]));
+                } else {
+#pragma unroll
+                    for (int v = 0; v < V; ++v)
+                        if (e0 + v < valid) gout[e0 + v] = y[v];
                 }
                 before += tot;
             }
@@ -155,6 +148,8 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
         }
 
         if (mt != 0 && !corrupt) {
+            // Every compute thread's reconstruction stores of this chunk come
+            // before any outlier store (the barrier orders them for the CTA).
             named_bar(1, kNW * 32);
             const uint32_t *gidx = reinterpret_cast<const uint32_t *>(a.in + stream_layout(a.n, a.block).record_off) +
                                    sm.info[s][6] + PW;
@@ -163,22 +158,13 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
                 const uint32_t val = staged ? rec[PW + mt + k] : gidx[mt + k];
                 const uint64_t e = (uint64_t)idx - (uint64_t)tile * kChunk;
                 if (idx >= (uint64_t)tile * kChunk && e < valid)
-                    sm.out[e] = __uint_as_float(val);
+                    gout[e] = __uint_as_float(val);
                 else
                     atomicOr(a.err, kErrCorrupt);
             }
-            named_bar(1, kNW * 32);
         }
         __syncwarp();
         if (ln == 0) mbar_arrive(&sm.empty[s]);
-
-        if (mt != 0 && !corrupt) {
-            const uint32_t n4 = valid / 4;
-            for (uint32_t j = tid; j < n4; j += kNW * 32)
-                __stcs(reinterpret_cast<float4 *>(gout) + j, reinterpret_cast<const float4 *>(sm.out)[j]);
-            for (uint32_t j = n4 * 4 + tid; j < valid; j += kNW * 32) gout[j] = sm.out[j];
-            named_bar(1, kNW * 32);  // the tile is free for the next chunk with outliers
-        }
     }
 }
 
@@ -257,7 +243,7 @@ __device__ void producer_warp(DecSmem &sm, const DecodeArgs &a, int ln) {
 }
 
 template <int V, int LPB>
-__global__ void __launch_bounds__(kThreads, 3) decode_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     DecSmem &sm = *reinterpret_cast<DecSmem *>(smem_raw);
     const int warp = threadIdx.x / 32, ln = threadIdx.x % 32;
@@ -283,7 +269,7 @@ cudaError_t launch_t(const DecodeArgs &a, int num_sms, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const uint64_t nc = (a.n + kChunk - 1) / kChunk;
     if (nc == 0) return cudaSuccess;
-    const uint64_t want = (uint64_t)num_sms * 3;
+    const uint64_t want = (uint64_t)num_sms * 4;
     const int grid = (int)(want < nc ? want : nc);
     decode_kernel<V, LPB><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
