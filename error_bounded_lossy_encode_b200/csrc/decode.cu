@@ -106,16 +106,31 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
                 const uint32_t mask = (w == 32u) ? kFull : ((1u << w) - 1u);
                 int32_t c[V];
                 uint32_t run = 0;
+                // Every word this lane reads lies in the staged record (widths
+                // checked above): one test for the lane instead of one per code.
+                const bool inside = ((bit0 + V * w) >> 5) + 1 < kRecWords - adj;
+                if (__all_sync(kFull, inside)) {
 #pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    const uint32_t b = bit0 + v * w;
-                    const uint32_t wd = b >> 5;
-                    const uint32_t zz = (wd + 1 < kRecWords - adj)
-                                            ? (__funnelshift_r(rec[wd], rec[wd + 1], b & 31u) & mask)
-                                            : 0u;
-                    const uint32_t d = (zz >> 1) ^ (0u - (zz & 1u));  // inverse zigzag
-                    run += d;
-                    c[v] = (int32_t)run;
+                    for (int v = 0; v < V; ++v) {
+                        const uint32_t b = bit0 + v * w;
+                        const uint32_t wd = b >> 5;
+                        const uint32_t zz = __funnelshift_r(rec[wd], rec[wd + 1], b & 31u) & mask;
+                        const uint32_t d = (zz >> 1) ^ (0u - (zz & 1u));  // inverse zigzag
+                        run += d;
+                        c[v] = (int32_t)run;
+                    }
+                } else {
+#pragma unroll
+                    for (int v = 0; v < V; ++v) {
+                        const uint32_t b = bit0 + v * w;
+                        const uint32_t wd = b >> 5;
+                        const uint32_t zz = (wd + 1 < kRecWords - adj)
+                                                ? (__funnelshift_r(rec[wd], rec[wd + 1], b & 31u) & mask)
+                                                : 0u;
+                        const uint32_t d = (zz >> 1) ^ (0u - (zz & 1u));  // inverse zigzag
+                        run += d;
+                        c[v] = (int32_t)run;
+                    }
                 }
                 uint32_t incl;
                 const uint32_t ex = group_scan_excl<LPB>(run, r, incl);
