@@ -54,6 +54,7 @@ constexpr int kThreads = (kNW + kLookbackWarps + 1) * 32;
 constexpr int kWindow = 10;               // look-back rows of 32 status words per round trip
 constexpr uint32_t kRing = 1536;          // packed words a compute warp can hold (3 worst-case tiles)
 constexpr uint32_t kWarpMax = kChunk / kNW;  // most words a warp packs for one tile
+static_assert(kRing >= 3 * kWarpMax, "one pending part must always leave room for the next");
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint64_t kInclBit = 1ull << 63;
 
@@ -548,7 +549,11 @@ __device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
         if (tile != 0) {  // the aggregate is already published by the compute warps
             // Start once this CTA has also computed its next tile: by then the
             // other CTAs have almost always published this tile's predecessors
-            // of the same wave, so the look-back rarely has to wait.
+            // of the same wave, so the look-back rarely has to wait.  This wait
+            // cannot close a cycle: a compute warp at iteration i + 1 never
+            // needs tile i written out, because with a single pending part of
+            // at most kWarpMax words a ring of 3 * kWarpMax words always has
+            // kWarpMax contiguous free words.
             if (!mbar_wait(&sm.computed[(i + 1) % kD], ((i + 1) / kD) & 1, a.wait_ns, a.err)) return;
             look_back(a, sm.st_cur, tile, -1, pack_status(0, 0, true), ln, exR, exM);
             if (ln == 0 && publish) st_relaxed_gpu(&sm.st_cur[tile], pack_status(exR + Rt, exM + MT, true));
