@@ -88,3 +88,41 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(E, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         E.lib()
+
+
+def test_product_path_never_touches_the_oracle():
+    """The library and its binding neither import, load nor execute anything
+    under oracle/: only the tests, the smoke check and the benchmark's CPU
+    legs may.  Python: no import of it and no string naming it outside
+    docstrings; C/CUDA: no reference to its symbols or files outside comments."""
+    import ast
+    import pathlib
+    import re
+
+    root = pathlib.Path(__file__).resolve().parents[1]
+    pkg = root / "error_bounded_lossy_encode_b200"
+    offenders = []
+    for path in pkg.rglob("*.py"):
+        tree = ast.parse(path.read_text())
+        docstrings = set()
+        for node in ast.walk(tree):
+            if isinstance(node, (ast.Module, ast.FunctionDef, ast.ClassDef, ast.AsyncFunctionDef)):
+                body = getattr(node, "body", [])
+                if body and isinstance(body[0], ast.Expr) and isinstance(getattr(body[0], "value", None), ast.Constant):
+                    docstrings.add(id(body[0].value))
+        for node in ast.walk(tree):
+            if isinstance(node, ast.Import) and any("oracle" in a.name for a in node.names):
+                offenders.append(f"{path.name}:{node.lineno} import")
+            if isinstance(node, ast.ImportFrom) and "oracle" in (node.module or ""):
+                offenders.append(f"{path.name}:{node.lineno} from-import")
+            if isinstance(node, ast.Constant) and isinstance(node.value, str) and id(node) not in docstrings \
+                    and re.search(r"oracle|eblc_oracle", node.value):
+                offenders.append(f"{path.name}:{node.lineno} string {node.value[:40]!r}")
+    pattern = re.compile(r"eblc_oracle|\borc_\w+|oracle/")
+    for path in list(pkg.rglob("*.cu")) + list(pkg.rglob("*.cuh")) + list(pkg.rglob("*.h")) + \
+            list((root / "include").rglob("*.h")):
+        text = re.sub(r"/\*.*?\*/", "", path.read_text(), flags=re.S)
+        for ln, line in enumerate(text.splitlines(), 1):
+            if pattern.search(line.split("//")[0]):
+                offenders.append(f"{path.name}:{ln}: {line.strip()}")
+    assert not offenders, offenders
