@@ -126,3 +126,43 @@ def test_product_path_never_touches_the_oracle():
             if pattern.search(line.split("//")[0]):
                 offenders.append(f"{path.name}:{ln}: {line.strip()}")
     assert not offenders, offenders
+
+
+def test_header_compiles_as_c99_and_links(tmp_path):
+    """A plain C program (C99, -Wall -Werror) includes the header, links
+    against the library and exercises the calls that need no GPU."""
+    import shutil
+    import subprocess
+
+    import error_bounded_lossy_encode_b200 as E
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    E.lib()  # fails loudly when the library is not built
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "eblc.h"
+int main(void) {
+    if (eblc_abi_version() != EBLC_ABI_VERSION) return 1;
+    if (strcmp(eblc_status_string(EBLC_OK), "ok") != 0) return 2;
+    eblc_plan_t plan = (eblc_plan_t)1;
+    int64_t dims[1] = {100};
+    if (eblc_plan_create(&plan, 1, dims, NULL, "block=48") != EBLC_UNSUPPORTED || plan != NULL) return 3;
+    if (eblc_plan_create(&plan, 0, dims, NULL, NULL) != EBLC_INVALID_ARG) return 4;
+    if (eblc_compress(NULL, NULL, NULL, NULL, 0, NULL, NULL) != EBLC_INVALID_ARG) return 5;
+    if (sizeof(eblc_sidecar_t) != 64 || sizeof(eblc_async_result_t) != 32) return 6;
+    eblc_plan_destroy(NULL);
+    puts("c abi ok");
+    return 0;
+}
+""")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(E.LIB_PATH)
+    inc = os.path.join(os.path.dirname(libdir), "include")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", inc, str(src), "-o", str(exe),
+                    "-L", libdir, "-leblc", "-Wl,-rpath," + libdir], check=True, capture_output=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, (r.returncode, r.stdout, r.stderr)
