@@ -668,8 +668,14 @@ cudaError_t launch_t(const EncodeArgs &a, int num_sms, cudaStream_t stream) {
                                        dim3(kThreads), params, smem, stream);
 }
 
-__global__ void finish_kernel(const FinishArgs f) {
+constexpr int kFinishThreads = 256;
+
+__global__ void __launch_bounds__(kFinishThreads) finish_kernel(const FinishArgs f) {
     const uint32_t err = *f.err;
+    if (err != 0u)
+        for (uint64_t j = threadIdx.x; j < f.status_words; j += kFinishThreads) f.status[j] = 0ull;
+    __syncthreads();  // every thread has read err before thread 0 clears it
+    if (threadIdx.x != 0) return;
     f.result[7] = err;
     *f.err = 0u;
     *f.epoch += 1u;
@@ -688,7 +694,7 @@ __global__ void finish_kernel(const FinishArgs f) {
 }  // namespace
 
 cudaError_t launch_finish(const FinishArgs &f, cudaStream_t stream) {
-    finish_kernel<<<1, 1, 0, stream>>>(f);
+    finish_kernel<<<1, kFinishThreads, 0, stream>>>(f);
     return cudaGetLastError();
 }
 

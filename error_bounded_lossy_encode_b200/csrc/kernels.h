@@ -43,15 +43,19 @@ struct EncodeArgs {
 };
 cudaError_t launch_encode(const EncodeArgs &a, int num_sms, cudaStream_t stream);
 
-// One thread, after the encoder on the same stream: result[7] = the call's
-// error word, which it then clears; advances the call counter; and, when
-// `user` is set, writes the caller's result record (compressed bytes,
-// payload words, outliers, status code).
+// After the encoder on the same stream: result[7] = the call's error word,
+// which it then clears; advances the call counter; when `user` is set,
+// writes the caller's result record (compressed bytes, payload words,
+// outliers, status code); and when the call failed (a wait that ran out
+// leaves look-back words behind) zeroes both look-back arrays, so the plan's
+// next call starts clean.
 struct FinishArgs {
     uint64_t *result;         // the encoder's result block (8 words)
     uint32_t *err;
     uint32_t *epoch;
     uint64_t *user;           // NULL, or 4 words: total, W, m, status | reserved << 32
+    uint64_t *status;         // both look-back arrays
+    uint64_t status_words;    // their total length
 };
 cudaError_t launch_finish(const FinishArgs &f, cudaStream_t stream);
 

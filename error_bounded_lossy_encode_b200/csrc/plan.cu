@@ -82,6 +82,8 @@ struct eblc_plan_s {
     uint64_t outlier_cap = 0;
     uint64_t wait_ns = 2000ull * 1000000ull;
     int64_t stall_tile = -1;
+    uint64_t stall_call = 0;        // the compress call (0-based) that stall_tile applies to
+    uint64_t calls = 0;             // compress calls enqueued so far
     Layout L{};
     uint64_t max_bytes = 0;
 
@@ -201,6 +203,9 @@ eblc_status_t parse_options(const char *options, eblc_plan_s *p, bool *timing) {
         } else if (key == "stall_tile") {
             if (!parse_int(val, &iv) || iv < -1) return EBLC_INVALID_ARG;
             p->stall_tile = iv;
+        } else if (key == "stall_call") {
+            if (!parse_int(val, &iv) || iv < 0) return EBLC_INVALID_ARG;
+            p->stall_call = (uint64_t)iv;
         } else {
             return EBLC_UNSUPPORTED;
         }
@@ -301,13 +306,13 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
     ea.err = &p->d_rb->err;
     ea.result = p->d_rb->result;
     ea.outlier_cap = p->outlier_cap;
-    ea.stall_tile = p->stall_tile;
+    ea.stall_tile = (p->calls++ == p->stall_call) ? p->stall_tile : -1;
     ea.wait_ns = p->wait_ns;
     timing_mark(p, st, true, "encode");
     eblc_status_t s = cuda_status(launch_encode(ea, p->num_sms, st), "encode launch");
     timing_mark(p, st, false, nullptr);
     if (s != EBLC_OK) return s;
-    FinishArgs fa{p->d_rb->result, &p->d_rb->err, &p->d_rb->epoch, d_user};
+    FinishArgs fa{p->d_rb->result, &p->d_rb->err, &p->d_rb->epoch, d_user, p->status, 2 * p->ntiles};
     if ((s = cuda_status(launch_finish(fa, st), "finish launch")) != EBLC_OK) return s;
     if (!d_user)
         s = cuda_status(cudaMemcpyAsync(p->h_rb, p->d_rb, sizeof(Readback), cudaMemcpyDeviceToHost, st), "readback");

@@ -157,9 +157,12 @@ EBLC_API const char *eblc_status_string(eblc_status_t status);
  *                    EBLC_CAPACITY
  *   timing=1         record per-kernel device times (eblc_plan_kernel_times)
  *   wait_ms=<t>      limit of device-side waits in milliseconds (default 2000)
- *   stall_tile=<t>   test hook: tile t of the next compress never publishes
+ *   stall_tile=<t>   test hook: tile t of one compress call never publishes
  *                    its scan value, so later tiles' waits run out and the
- *                    call returns EBLC_TIMEOUT (default off)
+ *                    call returns EBLC_TIMEOUT (default off); the plan's
+ *                    later calls are unaffected
+ *   stall_call=<k>   the compress call (0-based, counted per plan) that
+ *                    stall_tile applies to (default 0)
  * The plan allocates its device scratch here (cudaMalloc on the current
  * device).  *out is NULL on failure.
  */

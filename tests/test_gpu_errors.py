@@ -88,6 +88,47 @@ def test_lookback_timeout_is_reported(torch_cuda, orc):
         assert st == 0 and np.array_equal(got, orc.compress(x, 128, rel=1e-3))
 
 
+def test_plan_recovers_after_timeout(torch_cuda, orc):
+    """Call 0 succeeds, call 1 times out (tile 5 never publishes; later waits
+    give up, so some look-back words of the array call 2 will use are never
+    cleared), and calls 2 and 3 on the same plan, on other inputs, must again
+    produce the oracle's streams: a failed call's leftovers are cleared
+    before the next call."""
+    from tests.gpu_util import GpuCodec
+
+    xs = [WL.sine_noise(60 * 4096, k) for k in range(4)]
+    wants = [orc.compress(x, 128, rel=1e-3) for x in xs]
+    with GpuCodec(xs[0].size, 128, rel=1e-3, extra="stall_tile=5,stall_call=1,wait_ms=100") as g:
+        st, got, _ = g.compress_np(xs[0])
+        assert st == 0 and np.array_equal(got, wants[0])
+        st, _, _ = g.compress_np(xs[1])
+        assert st == E.EBLC_TIMEOUT
+        for k in (2, 3):
+            st, got, _ = g.compress_np(xs[k])
+            assert st == 0 and np.array_equal(got, wants[k]), k
+
+
+def test_async_timeout_reported_on_device(torch_cuda, orc):
+    import torch
+
+    from tests.gpu_util import GpuCodec
+
+    x_np = WL.sine_noise(60 * 4096, 7)
+    want = orc.compress(x_np, 128, rel=1e-3)
+    with GpuCodec(x_np.size, 128, rel=1e-3, extra="stall_tile=3,wait_ms=100") as g:
+        x = torch.from_numpy(x_np).cuda()
+        cap = g.lim["max_compressed_bytes"]
+        out = torch.zeros(cap, dtype=torch.uint8, device="cuda")
+        d_result = torch.zeros(32, dtype=torch.uint8, device="cuda")
+        ex = E.cuda_exec(torch.cuda.current_stream().cuda_stream)
+        for k, expect in enumerate((E.EBLC_TIMEOUT, E.EBLC_OK)):
+            assert E.eblc_compress_async(g.plan, ex, x.data_ptr(), out.data_ptr(), cap, d_result.data_ptr()) == 0
+            torch.cuda.synchronize()
+            r = E.async_result(d_result.cpu().numpy().tobytes())
+            assert r["status"] == expect, (k, r)
+        assert np.array_equal(out[: want.size].cpu().numpy(), want)
+
+
 def test_argument_errors(torch_cuda):
     st, plan = E.eblc_plan_create([1000], None, "rel=1e-3,block=64")
     assert st == 0
