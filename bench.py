@@ -158,6 +158,12 @@ def workload(name: str, elements: int | None = None, rel=None, abs_=None, block=
     return x, (block or blk), mode, bound
 
 
+def workload_config(args, n, block, mode, bound, world):
+    """The `config` both arms report for the same workload."""
+    return {"workload": args.workload if not args.elements else f"{args.workload}[:{n}]",
+            "n": int(n), "block": block, mode: bound, "parallelism": f"replicas{world}"}
+
+
 def options_string(block, mode, bound, timing=False):
     return f"{mode}={bound!r},block={block}" + (",timing=1" if timing else "")
 
@@ -233,8 +239,7 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": round(1e3 * elapsed / max(1, args.steps), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": args.workload, "n": int(min(x.size, CPU_SAMPLE_ELEMS)), "block": block,
-                       mode: bound, "sample_of_elements": int(x.size)},
+            "config": workload_config(args, x.size, block, mode, bound, world),
             "cpu_baseline": base,
             "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -455,10 +460,8 @@ def report(args, world, n, nbytes, t_comp, t_dec, t_comp_api, t_dec_api, total_i
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": args.workload if not args.elements else f"{args.workload}[:{n}]",
-                   "n": int(n), "block": block, mode: bound,
-                   "l2": "flushed (256 MiB write, untimed) before every compress and decompress call",
-                   "parallelism": f"replicas{world}"},
+        "config": dict(workload_config(args, n, block, mode, bound, world),
+                       l2="flushed (256 MiB write, untimed) before every compress and decompress call"),
         "compress_gbs": round(comp_gbs, 2),
         "decompress_gbs": round(dec_gbs, 2),
         "api_ms_per_step": {"compress": round(1e3 * t_comp_api / args.steps, 4),
