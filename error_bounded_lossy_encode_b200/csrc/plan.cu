@@ -156,7 +156,7 @@ std::string trim(const std::string &s) {
 
 eblc_status_t parse_options(const char *options, eblc_plan_s *p, bool *timing) {
     p->abs_mode = 0;
-    p->bound = 1e-4;  // provider default: the reference's default relative bound
+    p->bound = 1e-4;  // default relative bound ("Pipeline specialization internals", Priming)
     p->block = 128;
     *timing = false;
     if (!options) return EBLC_OK;
