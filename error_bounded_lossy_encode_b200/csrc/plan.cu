@@ -464,7 +464,7 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
     cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, p->device);
     cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device);
     if (major != 10 || minor != 0 || p->num_sms <= 0) {
-        EBLC_LOG("device %d is sm_%d%d; this build targets sm_100a", p->device, major, minor);
+        EBLC_LOG("device %d is sm_%d%d; libeblc is compiled for sm_100a only", p->device, major, minor);
         delete p;
         return EBLC_UNSUPPORTED;
     }
