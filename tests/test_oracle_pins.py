@@ -425,3 +425,60 @@ def test_golden_fixtures(orc):
         s = orc.compress(x, c["block"], **{c["mode"]: c["bound"]})
         assert s.size == c["total"]
         assert WL.sha256(s) == c["stream_sha256"], c["name"]
+
+
+# --------------------------------------------------------------------------------------
+# Property-based: random small arrays mixing ordinary values, huge and tiny magnitudes,
+# ties, signed zeros and non-finite values, over both bound modes and every block size
+# --------------------------------------------------------------------------------------
+
+def _fuzz_settings():
+    from hypothesis import HealthCheck, settings
+
+    return settings(max_examples=120, deadline=None, derandomize=True,
+                    suppress_health_check=[HealthCheck.too_slow, HealthCheck.data_too_large])
+
+
+def test_stream_invariants_fuzz(orc):
+    from hypothesis import given
+    from hypothesis import strategies as st
+
+    finite = st.floats(width=32, allow_nan=False, allow_infinity=False)
+    special = st.sampled_from([0.0, -0.0, float("nan"), float("inf"), float("-inf"), 1e-45, -1e-45, 2.0 ** 30,
+                               -(2.0 ** 31), 0.5, 1.5, 2.5, 1e38])
+    values = st.lists(st.one_of(finite, special, st.floats(-10, 10, width=32)), min_size=0, max_size=600)
+
+    @_fuzz_settings()
+    @given(values, st.sampled_from([32, 64, 128, 256]), st.sampled_from(["rel", "abs"]),
+           st.sampled_from([0.0, 1e-7, 1e-4, 1e-2, 0.25, 3.0, 1e30]))
+    def check(vals, block, mode, bound):
+        x = np.array(vals, dtype=np.float32)
+        s = orc.compress(x, block, **{mode: bound})
+        _check_stream(orc, x, s, block)
+
+    check()
+
+
+def test_stream_invariants_fuzz_multichunk(orc):
+    """Sizes across several 4096-element chunks and ragged tails, values from a
+    seeded mixture (smooth, noisy, spikes, specials), random bound and block."""
+    from hypothesis import given
+    from hypothesis import strategies as st
+
+    @_fuzz_settings()
+    @given(st.integers(0, 2 ** 32 - 1), st.sampled_from([1, 4095, 4096, 4097, 8191, 3 * 4096 + 17, 5 * 4096]),
+           st.sampled_from([32, 64, 128, 256]), st.sampled_from(["rel", "abs"]),
+           st.sampled_from([0.0, 1e-6, 1e-3, 0.1, 10.0]))
+    def check(seed, n, block, mode, bound):
+        rng = np.random.default_rng(seed)
+        t = np.arange(n)
+        x = np.sin(t / rng.uniform(5, 500)) * rng.uniform(0.1, 1e3) + rng.normal(0, rng.uniform(0, 1), n)
+        spikes = rng.random(n) < rng.uniform(0, 0.05)
+        x[spikes] = rng.uniform(-1e6, 1e6, int(spikes.sum()))
+        bad = rng.random(n) < 1e-3
+        x[bad] = rng.choice([np.nan, np.inf, -np.inf, 0.0, -0.0], int(bad.sum()))
+        x = x.astype(np.float32)
+        s = orc.compress(x, block, **{mode: bound})
+        _check_stream(orc, x, s, block)
+
+    check()
