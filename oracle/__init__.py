@@ -22,8 +22,10 @@ from dataclasses import dataclass
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "eblc_oracle.c")
-_LIB = os.path.join(_HERE, "liboracle.so")
+# EBLC_ORACLE_SRC points the tests at another copy of the source (the
+# planted-mistake tests build mutated copies in a temporary directory).
+_SRC = os.environ.get("EBLC_ORACLE_SRC") or os.path.join(_HERE, "eblc_oracle.c")
+_LIB = (_SRC[:-2] + ".so") if os.environ.get("EBLC_ORACLE_SRC") else os.path.join(_HERE, "liboracle.so")
 
 ERR_ARG, ERR_CAPACITY, ERR_OUTLIER_CAP, ERR_CORRUPT, ERR_NOMEM = -1, -2, -3, -4, -5
 CHUNK = 4096
