@@ -34,12 +34,12 @@ struct NoallocScratch {
     uint32_t range_counter;
     uint32_t pad[5];
     uint64_t result[8];
+    float range[4];          // vmin, vmax: zero when the range kernel does not run (n == 0)
     // written before being read within a call
-    float range[4];
     float2 partials[kMaxRangeParts];
     uint64_t status[2][kMaxTiles];
 };
-constexpr size_t kClearBytes = offsetof(NoallocScratch, range);
+constexpr size_t kClearBytes = offsetof(NoallocScratch, partials);
 
 static __device__ __align__(256) NoallocScratch g_noalloc_scratch;
 
@@ -84,9 +84,10 @@ extern "C" EBLC_API eblc_status_t eblc_compress_noalloc(const float *d_in, uint6
 
     int dev = 0, major = 0, minor = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return EBLC_CUDA_ERROR;
-    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return EBLC_CUDA_ERROR;
     if (major != 10 || minor != 0 || sms <= 0 || range_grid(sms) > kMaxRangeParts) return EBLC_UNSUPPORTED;
     NoallocScratch *S = nullptr;
     if (scratch_on_current_device(dev, &S) != cudaSuccess) return EBLC_CUDA_ERROR;

@@ -280,12 +280,14 @@ EBLC_API void eblc_plan_destroy(eblc_plan_t plan);
  *   compressed_bytes, h_sidecar  as for eblc_compress (h_sidecar may be NULL)
  * The scratch of the range and encode kernels is a file-scope __device__
  * array that every GPU that loads this library holds until the process
- * exits.  The first call on a device looks up that array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * exits.  The first call on a device does a one-time set-up: it looks up
+ * that array's device address (cudaGetSymbolAddress) with the device
+ * current.  Make that first call before any stream capture begins.
  * Every call on a device shares the array and each call clears what must
- * start at zero, so calls that overlap on the GPU (other streams, other
- * host threads) race: serialise them.  Like eblc_compress, the call
- * synchronises `stream` once at the end.
+ * start at zero (including the value range when n is 0), so calls that
+ * overlap on the GPU (other streams, other host threads) race: serialise
+ * them.  Like eblc_compress, the call ends by copying the result to the
+ * host and synchronising `stream`.
  */
 EBLC_API eblc_status_t eblc_compress_noalloc(const float *d_in, uint64_t n, uint32_t block, int abs_mode,
                                              double bound, void *d_out, size_t out_capacity, void *stream,
