@@ -22,8 +22,8 @@
 //               bulk async copies completing on mbarriers.
 // The reconstruction is stored straight from registers (128-bit coalesced
 // streaming stores); a chunk's outliers are then written over it in global
-// memory, after a barrier of the compute warps orders them behind every
-// reconstruction store of the chunk.
+// memory, after an mbarrier of the compute warps (bounded wait) orders them
+// behind every reconstruction store of the chunk.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -42,6 +42,7 @@ struct __align__(128) DecSmem {
     uint8_t width[kS][kChunk / 32];
     uint32_t info[kS][8];  // tile (or -1), valid, PW, mt, adj, staged, rec, corrupt
     uint64_t full[kS], empty[kS];
+    uint64_t stored;       // compute warps: a chunk's reconstruction stores are done (one phase per use)
 };
 
 template <int LPB>
@@ -65,6 +66,7 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
     constexpr int kEPL = kB / 32;  // payload words per unit of width for a full block
     const int g = ln / LPB, r = ln % LPB;
     const int tid = cw * 32 + ln;
+    uint32_t stored_uses = 0;  // phases of sm.stored this warp has waited for (the same for every warp)
 
     for (uint32_t i = 0;; ++i) {
         const int s = i % kS;
@@ -164,8 +166,15 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
 
         if (mt != 0 && !corrupt) {
             // Every compute thread's reconstruction stores of this chunk come
-            // before any outlier store (the barrier orders them for the CTA).
-            named_bar(1, kNW * 32);
+            // before any outlier store: each warp arrives (release) once its
+            // lanes' stores are done and waits (acquire) for all kNW warps.
+            // The wait is bounded like every other: a warp that gave up
+            // earlier never arrives, so the others record kErrTimeout and
+            // return instead of waiting for good.
+            __syncwarp();
+            if (ln == 0) mbar_arrive(&sm.stored);
+            if (!mbar_wait(&sm.stored, stored_uses & 1u, a.wait_ns, a.err)) return;
+            ++stored_uses;
             const uint32_t *gidx = reinterpret_cast<const uint32_t *>(a.in + stream_layout(a.n, a.block).record_off) +
                                    sm.info[s][6] + PW;
             for (uint32_t k = tid; k < mt; k += kNW * 32) {
@@ -267,6 +276,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeArgs a)
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kNW);
         }
+        mbar_init(&sm.stored, kNW);
         mbar_init_fence();
     }
     __syncthreads();
