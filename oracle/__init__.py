@@ -41,6 +41,21 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+_OMP_SRC = os.path.join(_HERE, "eblc_oracle_omp.c")
+_OMP_LIB = os.path.join(_HERE, "liboracle_omp.so")
+
+
+def build_omp(force: bool = False) -> str:
+    """Compile the all-core build (eblc_oracle_omp.c: the oracle's own steps,
+    run over chunks with OpenMP; the benchmark's all-core CPU baseline)."""
+    newest = max(os.path.getmtime(_OMP_SRC), os.path.getmtime(_SRC))
+    if force or not os.path.exists(_OMP_LIB) or os.path.getmtime(_OMP_LIB) < newest:
+        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+               "-fPIC", "-shared", "-I", os.path.dirname(_SRC), "-o", _OMP_LIB, _OMP_SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _OMP_LIB
+
+
 class _Header(ctypes.Structure):
     _fields_ = [(k, ctypes.c_uint32) for k in ("magic", "version", "flags", "block", "chunk", "pad")] + \
                [(k, ctypes.c_uint64) for k in ("n", "nb", "nc", "W", "m", "total")] + \
@@ -212,3 +227,52 @@ def block_codes(x, block: int, inv2eb) -> tuple[np.ndarray, np.ndarray]:
     w = np.zeros(max(1, nb), np.uint8)
     lib().orc_block_codes(_ptr(x), x.size, block, float(np.float32(inv2eb)), _ptr(z), _ptr(w))
     return z[: x.size], w[:nb]
+
+
+_omp = None
+
+
+def _omp_lib():
+    global _omp
+    if _omp is None:
+        L = ctypes.CDLL(build_omp())
+        P, u64, u32, dbl = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_uint32, ctypes.c_double
+        L.orc_compress_omp.argtypes = [P, u64, u32, ctypes.c_int, dbl, u64, P, u64]
+        L.orc_compress_omp.restype = ctypes.c_int64
+        L.orc_decompress_omp.argtypes = [P, u64, P, u64]
+        L.orc_decompress_omp.restype = ctypes.c_int
+        L.orc_omp_threads.argtypes = []
+        L.orc_omp_threads.restype = ctypes.c_int
+        _omp = L
+    return _omp
+
+
+def omp_threads() -> int:
+    """Threads the all-core build uses (OpenMP's default: the cores this
+    process may run on, or OMP_NUM_THREADS)."""
+    return int(_omp_lib().orc_omp_threads())
+
+
+def compress_omp(x, block: int = 128, *, rel: float | None = None, abs: float | None = None):
+    """compress() on all host cores; the stream is byte-identical."""
+    x = _f32(x).reshape(-1)
+    if (rel is None) == (abs is None):
+        raise ValueError("exactly one of rel / abs")
+    abs_mode = abs is not None
+    need = max_compressed_bytes(x.size, block)
+    out = np.zeros(max(need, 1), np.uint8)
+    rc = _omp_lib().orc_compress_omp(_ptr(x), x.size, block, int(abs_mode), float(abs if abs_mode else rel),
+                                     x.size, _ptr(out), need)
+    if rc < 0:
+        raise OracleError(int(rc))
+    return out[:rc].copy()
+
+
+def decompress_omp(stream, n: int) -> np.ndarray:
+    """decompress() on all host cores."""
+    s = np.ascontiguousarray(stream, dtype=np.uint8)
+    out = np.zeros(max(n, 1), np.float32)
+    rc = _omp_lib().orc_decompress_omp(_ptr(s), s.size, _ptr(out), n)
+    if rc != 0:
+        raise OracleError(rc)
+    return out[:n]
