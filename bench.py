@@ -12,14 +12,19 @@ timing is the max over ranks.
 
 Printed JSON line (rank 0):
   value        GB/s of float32 input per compress + decompress round trip,
-               device-resident input, CUDA events around the library calls;
-               the L2 is flushed (256 MiB write) before every call and the
-               flush is not timed
+               device-resident input: CUDA events on the call's stream around
+               each full API call (eblc_compress including its closing
+               synchronisation, eblc_decompress), median step of --steps
+               (best step in value_best); the L2 is flushed (256 MiB write)
+               before every call and the flush is not timed
   e2e          the same through the HOST execution kind (host buffers,
                host<->device copies inside the timed region)
   roofline     the dominant kernel against the measured copy bandwidth
-  cpu_baseline the CPU oracle on a bounded sample of the workload
---impl reference times the CPU oracle itself (the only reference there is).
+  cpu_baseline the plain single-threaded CPU oracle on a bounded sample of the
+               workload; cpu_baseline_all_cores the same oracle steps run over
+               chunks on all host cores (OpenMP build); host names the CPU
+--impl reference times the plain CPU oracle itself (the only reference there
+is) on the whole workload, with the same config as this arm.
 """
 from __future__ import annotations
 
@@ -161,7 +166,26 @@ def workload(name: str, elements: int | None = None, rel=None, abs_=None, block=
 def workload_config(args, n, block, mode, bound, world):
     """The `config` both arms report for the same workload."""
     return {"workload": args.workload if not args.elements else f"{args.workload}[:{n}]",
-            "n": int(n), "block": block, mode: bound, "parallelism": f"replicas{world}"}
+            "n": int(n), "block": block, mode: bound, "parallelism": f"replicas{world}",
+            "l2": "flushed (256 MiB write, untimed) before every GPU compress and decompress call"}
+
+
+def host_info():
+    """CPU model and the cores this process may run on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        cores = os.cpu_count()
+    return {"cpu_model": model, "cores_available": cores}
 
 
 def options_string(block, mode, bound, timing=False):
@@ -203,44 +227,69 @@ def profiled_traffic(kernel: str, workload_name: str):
 # ----------------------------------------------------------------------------------------------
 # CPU oracle legs
 
-def cpu_oracle_sample(x, block, mode, bound, repeats=1):
+def cpu_oracle_sample(x, block, mode, bound, repeats=1, all_cores=False, elems=CPU_SAMPLE_ELEMS):
+    """Time the CPU oracle (compress + decompress) on the first `elems`
+    elements: the plain single-threaded oracle, or (all_cores) the OpenMP
+    build of the same steps."""
     import oracle
 
     oracle.build()
-    s = x[:CPU_SAMPLE_ELEMS]
+    comp, decomp = (oracle.compress_omp, oracle.decompress_omp) if all_cores else \
+        (oracle.compress, oracle.decompress)
+    s = x[:elems]
     t_c = t_d = 0.0
     for _ in range(repeats):
         t0 = time.perf_counter()
-        stream = oracle.compress(s, block, **{mode: bound})
+        stream = comp(s, block, **{mode: bound})
         t1 = time.perf_counter()
-        oracle.decompress(stream, s.size)
+        decomp(stream, s.size)
         t2 = time.perf_counter()
         t_c += t1 - t0
         t_d += t2 - t1
     gbs = repeats * 4 * s.size / (t_c + t_d) / 1e9
-    return {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {s.size} elements ({4 * s.size >> 20} MiB) of the workload, compress+decompress, "
-                      f"single-threaded plain C oracle",
+    cores = oracle.omp_threads() if all_cores else 1
+    what = f"the oracle's steps run over chunks with OpenMP on {cores} threads" if all_cores else \
+        "single-threaded plain C oracle"
+    part = "the whole workload" if s.size == x.size else f"first {s.size} elements ({4 * s.size >> 20} MiB) of the workload"
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle" if not all_cores else "oracle (all-core OpenMP build)",
+            "sample": f"{part}, compress+decompress, {what}",
             "compress_gbs": round(repeats * 4 * s.size / t_c / 1e9, 4),
             "decompress_gbs": round(repeats * 4 * s.size / t_d / 1e9, 4)}
 
 
+REFERENCE_BUDGET_S = 150.0  # wall-time budget of the reference arm's timed steps
+
+
 def run_reference(args):
+    """The plain CPU oracle, timed on this arm's workload and config.  Each
+    step compresses and decompresses the whole workload when the steps fit
+    the time budget (estimated from one warm-up on a 2^22-element sample),
+    else a leading sample, which the config then names."""
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
     x, block, mode, bound = workload(args.workload, args.elements, args.rel, args.abs, args.block)
-    for _ in range(args.warmup):
-        cpu_oracle_sample(x, block, mode, bound)
+    probe = cpu_oracle_sample(x, block, mode, bound, elems=1 << 22)
+    est_step_s = 4.0 * x.size / (probe["value"] * 1e9)
+    elems = x.size if est_step_s * args.steps <= REFERENCE_BUDGET_S else \
+        max(1 << 22, int(REFERENCE_BUDGET_S / args.steps * probe["value"] * 1e9 / 4) // 4096 * 4096)
+    warm = args.warmup if est_step_s * (args.steps + args.warmup) <= 1.5 * REFERENCE_BUDGET_S else 1
+    for _ in range(warm):
+        cpu_oracle_sample(x, block, mode, bound, elems=min(elems, 1 << 22))
     t0 = time.perf_counter()
-    base = cpu_oracle_sample(x, block, mode, bound, repeats=args.steps)
+    base = cpu_oracle_sample(x, block, mode, bound, repeats=args.steps, elems=elems)
     elapsed = time.perf_counter() - t0
+    config = workload_config(args, x.size, block, mode, bound, world)
+    if elems < x.size:
+        config = dict(config, workload=f"{config['workload']}[:{elems}]", n=int(elems))
     line = {"metric": METRIC, "value": base["value"], "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * elapsed / max(1, args.steps), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "impl": "reference",
-            "config": workload_config(args, x.size, block, mode, bound, world),
+            "config": config,
             "cpu_baseline": base,
+            "host": host_info(),
             "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -324,21 +373,25 @@ def run_ours(args):
         dist.barrier()
     clk = clocks.stop() if clocks else None
 
-    # device time of the library calls (first launch to last device operation)
-    t_comp = sum(r[5]["compress_call"] for r in recs) / 1e3
-    t_dec = sum(r[5]["decompress_call"] for r in recs) / 1e3
-    # the same bracketed by torch events from Python (includes host return latency)
-    t_comp_api = sum(r[0].elapsed_time(r[1]) for r in recs) / 1e3
-    t_dec_api = sum(r[2].elapsed_time(r[3]) for r in recs) / 1e3
+    # CUDA events on the call's stream around each full API call (compress
+    # includes its closing synchronisation and readback): per step, seconds
+    comp_api = [r[0].elapsed_time(r[1]) / 1e3 for r in recs]
+    dec_api = [r[2].elapsed_time(r[3]) / 1e3 for r in recs]
+    steps_api = [c + d for c, d in zip(comp_api, dec_api)]
+    # the library's own events, first launch to last device operation of the call
+    comp_dev = [r[5]["compress_call"] / 1e3 for r in recs]
+    dec_dev = [r[5]["decompress_call"] / 1e3 for r in recs]
     nbytes = recs[-1][4]
     kern = {}
     for r in recs:
         for k, ms in r[5].items():
             if not k.endswith("_call"):
                 kern.setdefault(k, []).append(ms)
-    t_comp, t_dec, t_comp_api, t_dec_api = max_over_ranks([t_comp, t_dec, t_comp_api, t_dec_api], world, dev)
-    total_in_bytes = sum_over_ranks([4.0 * n * args.steps], world, dev)[0]
-    step_s = (t_comp + t_dec) / args.steps
+    med = lambda v: float(np.median(v))
+    T = dict(zip(["step", "step_best", "comp", "dec", "comp_dev", "dec_dev"],
+                 max_over_ranks([med(steps_api), min(steps_api), med(comp_api), med(dec_api), med(comp_dev),
+                                 med(dec_dev)], world, dev)))
+    step_bytes = sum_over_ranks([4.0 * n], world, dev)[0]
 
     graph = run_graph_compress(E, plan, x, out, cap, flush, nbytes, args, world, dev)
 
@@ -347,8 +400,8 @@ def run_ours(args):
     if not args.no_e2e:
         e2e = run_e2e(E, plan, x_np, cap, args, world, dev)
     if rank == 0:
-        report(args, world, n, nbytes, t_comp, t_dec, t_comp_api, t_dec_api, total_in_bytes, step_s, kern, e2e,
-               launches_per_step, clk, x_np, block, mode, bound, graph)
+        report(args, world, n, nbytes, T, step_bytes, kern, e2e, launches_per_step, clk, x_np, block, mode, bound,
+               graph)
     E.eblc_plan_destroy(plan)
     if world > 1:
         import torch.distributed as dist
@@ -432,45 +485,47 @@ def run_e2e(E, plan, x_np, cap, args, world, dev):
                    "from each call's input copy to its output copy, max over ranks"}
 
 
-def report(args, world, n, nbytes, t_comp, t_dec, t_comp_api, t_dec_api, total_in_bytes, step_s, kern, e2e,
-           launches_per_step, clk, x_np, block, mode, bound, graph=None):
+def report(args, world, n, nbytes, T, step_bytes, kern, e2e, launches_per_step, clk, x_np, block, mode, bound,
+           graph=None):
     peak, peak_kind = measured_peak()
     ratio = 4.0 * n / nbytes
-    comp_gbs = 4.0 * n * args.steps / t_comp / 1e9
-    dec_gbs = 4.0 * n * args.steps / t_dec / 1e9
     algo = {"range": 4.0 * n, "encode": 4.0 * n + nbytes, "decode": 4.0 * n + nbytes}
     kstats = {}
     for k, v in kern.items():
         avg_ms = float(np.mean(v))
         ach = algo[k] / (avg_ms / 1e3) / 1e9
-        kstats[k] = {"avg_ms": round(avg_ms, 4), "launches": len(v), "algorithmic_bytes": int(algo[k]),
-                     "achieved_gbs": round(ach, 1), "frac_of_measured_peak": round(ach / peak, 4)}
+        kstats[k] = {"avg_ms": round(avg_ms, 4), "median_ms": round(float(np.median(v)), 4), "launches": len(v),
+                     "algorithmic_bytes": int(algo[k]), "achieved_gbs": round(ach, 1),
+                     "frac_of_measured_peak": round(ach / peak, 4)}
     dom = max(kstats, key=lambda k: kstats[k]["avg_ms"])
     traffic = profiled_traffic(dom, args.workload)
     line = {
         "metric": METRIC,
-        "value": round(total_in_bytes / (t_comp + t_dec) / 1e9, 2),
+        "value": round(step_bytes / T["step"] / 1e9, 2),
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": max(3, args.warmup),
-        "ms_per_step": round(1e3 * step_s, 4),
+        "ms_per_step": round(1e3 * T["step"], 4),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": dict(workload_config(args, n, block, mode, bound, world),
-                       l2="flushed (256 MiB write, untimed) before every compress and decompress call"),
-        "compress_gbs": round(comp_gbs, 2),
-        "decompress_gbs": round(dec_gbs, 2),
-        "api_ms_per_step": {"compress": round(1e3 * t_comp_api / args.steps, 4),
-                            "decompress": round(1e3 * t_dec_api / args.steps, 4)},
+        "config": workload_config(args, n, block, mode, bound, world),
+        "timing": "CUDA events on the call's stream around each full API call (compress includes its closing "
+                  "synchronisation); median step, max over ranks",
+        "value_best": round(step_bytes / T["step_best"] / 1e9, 2),
+        "compress_gbs": round(4.0 * n / T["comp"] / 1e9, 2),
+        "decompress_gbs": round(4.0 * n / T["dec"] / 1e9, 2),
+        "api_ms_per_step": {"compress": round(1e3 * T["comp"], 4), "decompress": round(1e3 * T["dec"], 4)},
+        "device_ms_per_step": {"compress": round(1e3 * T["comp_dev"], 4), "decompress": round(1e3 * T["dec_dev"], 4),
+                               "what": "library events: first launch to the last device operation of the call"},
         "ratio": round(ratio, 4),
         "stream_bytes": int(nbytes),
-        "hbm_frac_8tbs": {"compress": round((4.0 * n + nbytes) * args.steps / t_comp / 8e12, 4),
-                          "decompress": round((4.0 * n + nbytes) * args.steps / t_dec / 8e12, 4),
-                          "compress_required_bytes": round((8.0 * n + nbytes) * args.steps / t_comp / 8e12, 4)
+        "hbm_frac_8tbs": {"compress": round((4.0 * n + nbytes) / T["comp"] / 8e12, 4),
+                          "decompress": round((4.0 * n + nbytes) / T["dec"] / 8e12, 4),
+                          "compress_required_bytes": round((8.0 * n + nbytes) / T["comp"] / 8e12, 4)
                           if mode == "rel" else None},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": kstats[dom]["achieved_gbs"], "peak": peak,
                      "peak_kind": f"{peak_kind} copy bandwidth", "unit": "GB/s",
@@ -481,8 +536,14 @@ def report(args, world, n, nbytes, t_comp, t_dec, t_comp_api, t_dec_api, total_i
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if n <= (1 << 22):
+        line["note"] = ("input fits in L2 and each call is a few tens of microseconds: the synchronous compress is "
+                        "bound by launch and host synchronisation latency, not HBM (graph_compress shows the "
+                        "sync-free form)")
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(x_np, block, mode, bound)
+        line["cpu_baseline_all_cores"] = cpu_oracle_sample(x_np, block, mode, bound, all_cores=True)
+        line["host"] = host_info()
     print(json.dumps(line), flush=True)
 
 

@@ -72,17 +72,18 @@ class _Args:
 
 def test_report_line_contract(monkeypatch):
     """One JSON line with every key the benchmark contract names; value is the
-    whole job's input bytes over the slowest rank's compress + decompress time."""
+    whole job's input bytes of one step over the slowest rank's median step
+    (compress + decompress API calls), value_best over its best step."""
     n, nbytes, world = 1 << 20, 600_000, 2
-    t_comp, t_dec = 0.004, 0.002
+    T = {"step": 0.006, "step_best": 0.005, "comp": 0.004, "dec": 0.002, "comp_dev": 0.0035, "dec_dev": 0.0018}
     kern = {"range": [0.1] * 4, "encode": [0.6] * 4, "decode": [0.5] * 4}
     e2e = {"value": 12.0, "unit": "GB/s", "h2d_bytes_per_step": 4 * n + nbytes, "d2h_bytes_per_step": nbytes + 4 * n}
     clk = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": [], "samples": 3}
-    total = 4.0 * n * _Args.steps * world
+    step_bytes = 4.0 * n * world
     buf = io.StringIO()
     with redirect_stdout(buf):
-        bench.report(_Args, world, n, nbytes, t_comp, t_dec, t_comp, t_dec, total, (t_comp + t_dec) / _Args.steps,
-                     kern, e2e, 3, clk, np.zeros(n, np.float32), 64, "rel", 1e-3)
+        bench.report(_Args, world, n, nbytes, T, step_bytes, kern, e2e, 3, clk, np.zeros(n, np.float32), 64, "rel",
+                     1e-3)
     lines = [ln for ln in buf.getvalue().splitlines() if ln.strip()]
     assert len(lines) == 1
     d = json.loads(lines[0])
@@ -90,7 +91,10 @@ def test_report_line_contract(monkeypatch):
               "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks"):
         assert k in d, k
     assert d["n_gpus"] == world and d["scaling"] == "weak" and d["higher_is_better"] is True
-    assert d["value"] == pytest.approx(total / (t_comp + t_dec) / 1e9, rel=1e-3)
+    assert d["value"] == pytest.approx(step_bytes / T["step"] / 1e9, abs=0.006)
+    assert d["value_best"] == pytest.approx(step_bytes / T["step_best"] / 1e9, abs=0.006)
+    assert d["ms_per_step"] == pytest.approx(1e3 * T["step"], rel=1e-3)
+    assert "l2" in d["config"]
     assert d["config"]["workload"] == "field512cube_spikes"
     r = d["roofline"]
     assert r["bound"] == "hbm" and r["kernel"] == "encode" and r["unit"] == "GB/s"
@@ -106,3 +110,17 @@ def test_reference_arm_other_ranks_exit_quietly(monkeypatch):
     with redirect_stdout(buf):
         assert bench.run_reference(_Args) == 0
     assert buf.getvalue() == ""
+
+
+def test_both_arms_report_the_same_config():
+    """The reference arm times the plain oracle on this arm's workload: its
+    config is the one this arm prints (same workload, n, block, bound)."""
+    a = bench.workload_config(_Args, 1 << 20, 64, "rel", 1e-3, 1)
+    b = bench.workload_config(_Args, 1 << 20, 64, "rel", 1e-3, 1)
+    assert a == b and a["workload"] == "field512cube_spikes" and a["n"] == 1 << 20
+
+
+def test_host_info_names_cpu_and_cores():
+    h = bench.host_info()
+    assert h["cores_available"] >= 1
+    assert "cpu_model" in h
