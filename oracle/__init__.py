@@ -61,7 +61,8 @@ class _Header(ctypes.Structure):
                [(k, ctypes.c_uint64) for k in ("n", "nb", "nc", "W", "m", "total")] + \
                [("eb", ctypes.c_double), ("bound", ctypes.c_double)] + \
                [(k, ctypes.c_float) for k in ("inv2eb", "step", "vmin", "vmax")] + \
-               [(k, ctypes.c_uint64) for k in ("width_off", "index_off", "record_off")]
+               [(k, ctypes.c_uint64) for k in ("width_off", "index_off", "record_off")] + \
+               [("dims", ctypes.c_uint64 * 3)]
 
 
 _lib = None
@@ -95,8 +96,18 @@ def lib():
         L.orc_max_compressed_bytes.restype = u64
         L.orc_compress.argtypes = [P, u64, u32, ctypes.c_int, dbl, u64, P, u64]
         L.orc_compress.restype = ctypes.c_int64
+        L.orc_compress_range.argtypes = [P, u64, u32, dbl, flt, flt, u64, P, u64]
+        L.orc_compress_range.restype = ctypes.c_int64
         L.orc_parse_header.argtypes = [P, u64, ctypes.POINTER(_Header)]
         L.orc_parse_header.restype = ctypes.c_int
+        L.orc_compress_lorenzo.argtypes = [P, ctypes.c_int, P, u32, ctypes.c_int, dbl, u64, P, u64]
+        L.orc_compress_lorenzo.restype = ctypes.c_int64
+        L.orc_nd_edges.argtypes = [ctypes.c_int, u32, P, P]
+        L.orc_nd_edges.restype = ctypes.c_int
+        L.orc_lorenzo_block.argtypes = [P, P, P]
+        L.orc_lorenzo_block.restype = None
+        L.orc_unlorenzo_block.argtypes = [P, P, P]
+        L.orc_unlorenzo_block.restype = None
         L.orc_decompress.argtypes = [P, u64, P, u64]
         L.orc_decompress.restype = ctypes.c_int
         L.orc_block_codes.argtypes = [P, u64, u32, flt, P, P]
@@ -196,6 +207,21 @@ def compress(x, block: int = 128, *, rel: float | None = None, abs: float | None
     return out[:rc].copy()
 
 
+def compress_range(x, block: int, rel: float, vmin: float, vmax: float, *, outlier_cap: int | None = None):
+    """compress() of one part of a larger array under the relative bound of
+    the whole: eb = rel * (vmax - vmin) with the given range (see
+    orc_compress_range)."""
+    x = _f32(x).reshape(-1)
+    cap = x.size if outlier_cap is None else int(outlier_cap)
+    need = max_compressed_bytes(x.size, block, cap)
+    out = np.zeros(max(need, 1), np.uint8)
+    rc = lib().orc_compress_range(_ptr(x), x.size, block, float(rel), float(np.float32(vmin)),
+                                  float(np.float32(vmax)), cap, _ptr(out), need)
+    if rc < 0:
+        raise OracleError(int(rc))
+    return out[:rc].copy()
+
+
 class OracleError(RuntimeError):
     def __init__(self, code: int):
         super().__init__(f"oracle error {code}")
@@ -208,7 +234,56 @@ def parse_header(stream) -> dict:
     rc = lib().orc_parse_header(_ptr(s) if s.size else 0, s.size, ctypes.byref(h))
     if rc != 0:
         raise OracleError(rc)
-    return {k: getattr(h, k) for k, _ in _Header._fields_}
+    d = {k: getattr(h, k) for k, _ in _Header._fields_}
+    d["dims"] = tuple(int(v) for v in h.dims)
+    return d
+
+
+def nd_edges(rank: int, block: int):
+    """(block edges, brick edges), each (z, y, x), of the multi-dimensional
+    Lorenzo layout, or None when rank / block is not supported."""
+    be, ce = np.zeros(3, np.uint32), np.zeros(3, np.uint32)
+    if not lib().orc_nd_edges(rank, block, _ptr(be), _ptr(ce)):
+        return None
+    return tuple(int(v) for v in be), tuple(int(v) for v in ce)
+
+
+def lorenzo_block(q, be) -> np.ndarray:
+    """Lorenzo residuals of one block (codes in C order, edges be), int32 modulo 2^32."""
+    q = np.ascontiguousarray(q, dtype=np.int32).reshape(-1)
+    e = np.ascontiguousarray(be, dtype=np.uint32)
+    d = np.zeros(q.size, np.int32)
+    lib().orc_lorenzo_block(_ptr(q), _ptr(e), _ptr(d))
+    return d
+
+
+def unlorenzo_block(d, be) -> np.ndarray:
+    d = np.ascontiguousarray(d, dtype=np.int32).reshape(-1)
+    e = np.ascontiguousarray(be, dtype=np.uint32)
+    q = np.zeros(d.size, np.int32)
+    lib().orc_unlorenzo_block(_ptr(d), _ptr(e), _ptr(q))
+    return q
+
+
+def compress_lorenzo(x, block: int = 64, *, rel: float | None = None, abs: float | None = None,
+                     outlier_cap: int | None = None):
+    """compress() with the multi-dimensional Lorenzo predictor over x's own
+    dims (x of shape (Z, Y, X) or (Y, X); see orc_compress_lorenzo)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.ndim not in (2, 3):
+        raise ValueError("x must be 2-D or 3-D")
+    if (rel is None) == (abs is None):
+        raise ValueError("exactly one of rel / abs")
+    dims = np.array((1,) + x.shape if x.ndim == 2 else x.shape, np.uint64)
+    abs_mode = abs is not None
+    cap = x.size if outlier_cap is None else int(outlier_cap)
+    need = max_compressed_bytes(x.size, block, cap)
+    out = np.zeros(max(need, 1), np.uint8)
+    rc = lib().orc_compress_lorenzo(_ptr(x), x.ndim, _ptr(dims), block, int(abs_mode),
+                                    float(abs if abs_mode else rel), cap, _ptr(out), need)
+    if rc < 0:
+        raise OracleError(int(rc))
+    return out[:rc].copy()
 
 
 def decompress(stream, n: int) -> np.ndarray:

@@ -80,6 +80,7 @@
 #define ORC_CHUNK 4096u
 #define ORC_HEADER_BYTES 128u
 #define ORC_FLAG_ABS 1u
+#define ORC_FLAG_LORENZO_ND 2u    /* 2-D / 3-D Lorenzo over the array's own dims */
 
 /* error codes returned as negative values */
 #define ORC_ERR_ARG (-1)
@@ -273,16 +274,23 @@ uint64_t orc_max_compressed_bytes(uint64_t n, uint32_t block, uint64_t outlier_c
 
 /* ------------------------------------------------------------------------ */
 /* Compress x[0..n) into out[0..out_cap).  Returns the stream length, or a
- * negative ORC_ERR_* code.  More outliers than outlier_cap is an error.     */
-int64_t orc_compress(const float *x, uint64_t n, uint32_t block, int abs_mode, double bound,
-                     uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
+ * negative ORC_ERR_* code.  More outliers than outlier_cap is an error.
+ * `range` (relative bound only): NULL to take the value range of x itself
+ * (step 1), else {vmin, vmax} given by the caller.                         */
+static int64_t compress_with(const float *x, uint64_t n, uint32_t block, int abs_mode, double bound,
+                             const float *range, uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
     if (!block_ok(block) || !(bound >= 0.0) || !isfinite(bound)) return ORC_ERR_ARG;
     if (n > ORC_MAX_N) return ORC_ERR_ARG;
     if (fegetround() != FE_TONEAREST) return ORC_ERR_ARG;
 
     /* steps 1-2 */
     float vmin = 0.0f, vmax = 0.0f;
-    if (!abs_mode) orc_value_range(x, n, &vmin, &vmax);
+    if (!abs_mode && range) {
+        vmin = range[0] + 0.0f;
+        vmax = range[1] + 0.0f;
+    } else if (!abs_mode) {
+        orc_value_range(x, n, &vmin, &vmax);
+    }
     double eb;
     float inv2eb, step;
     orc_resolve_bound(abs_mode, bound, vmin, vmax, &eb, &inv2eb, &step);
@@ -398,6 +406,228 @@ int64_t orc_compress(const float *x, uint64_t n, uint32_t block, int abs_mode, d
     return (int64_t)L.total;
 }
 
+int64_t orc_compress(const float *x, uint64_t n, uint32_t block, int abs_mode, double bound,
+                     uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
+    return compress_with(x, n, block, abs_mode, bound, NULL, outlier_cap, out, out_cap);
+}
+
+/* One contiguous part of a larger array, coded under the relative bound of
+ * the whole: eb = rel * (vmax - vmin) with the whole array's value range
+ * {vmin, vmax} given by the caller instead of the part's own ([SPEC]
+ * Priming: the bound is resolved from a value range before any code is
+ * produced; "DevitoComp provider interface", Validating a private provider:
+ * the provider runs under an MPI-run consumer, one part of the domain per
+ * process).  vmin <= vmax, both finite, else ORC_ERR_ARG.  With the part's
+ * own range this is orc_compress.                                           */
+int64_t orc_compress_range(const float *x, uint64_t n, uint32_t block, double rel, float vmin, float vmax,
+                           uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
+    if (!isfinite(vmin) || !isfinite(vmax) || !(vmin <= vmax)) return ORC_ERR_ARG;
+    const float range[2] = {vmin, vmax};
+    return compress_with(x, n, block, 0, rel, range, outlier_cap, out, out_cap);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Multi-dimensional Lorenzo ([SPEC] Roles and strategies: a RegionLocal
+ * predictor is one whose values may depend on others within a fixed logical
+ * region, with no dependency across regions; the 1-D Lorenzo predictor with
+ * region reset is the one the pages print).  Reading for 2-D / 3-D data
+ * (the pages print no multi-dimensional predictor): the region is a block of
+ * the array's own dims -- bz x by x bx elements -- and the predictor is the
+ * classical Lorenzo stencil over the quantization codes, with every
+ * neighbour outside the block taken as 0 (the region reset):
+ *   d(i,j,k) = sum over a,b,c in {0,1} of (-1)^(a+b+c) q(i-a, j-b, k-c),
+ * i.e. the first difference along x, then y, then z.  Its inverse is the
+ * inclusive prefix sum along each axis of the block.  d is taken modulo
+ * 2^32 (two's complement), so the inverse is exact even where a sum of
+ * eight codes would not fit in 32 bits.
+ *
+ * Layout reading: a chunk is a brick of 16 x 16 x 16 elements (3-D) or
+ * 64 x 64 (2-D), the array's dims must be multiples of the brick, bricks are
+ * taken in C order over the brick grid, blocks in C order within a brick,
+ * codes in C order within a block; the header's bytes 96..119 hold Z, Y, X
+ * (Z = 1 for 2-D).  Outlier indices are the elements' C-order indices in
+ * the whole array, ascending within each brick.  Blocks: 64 -> 4x4x4 (3-D)
+ * or 8x8 (2-D); 256 -> 4x8x8 (3-D) or 16x16 (2-D).                        */
+int orc_nd_edges(int rank, uint32_t block, uint32_t be[3], uint32_t ce[3]) {
+    if (rank == 3) {
+        ce[0] = ce[1] = ce[2] = 16;
+        if (block == 64) { be[0] = 4; be[1] = 4; be[2] = 4; return 1; }
+        if (block == 256) { be[0] = 4; be[1] = 8; be[2] = 8; return 1; }
+    } else if (rank == 2) {
+        ce[0] = 1; ce[1] = ce[2] = 64;
+        if (block == 64) { be[0] = 1; be[1] = 8; be[2] = 8; return 1; }
+        if (block == 256) { be[0] = 1; be[1] = 16; be[2] = 16; return 1; }
+    }
+    return 0;
+}
+
+/* Flat C-order index of element e (block order) of block `b` (brick order)
+ * for dims d[3], block edges be[3], brick edges ce[3].                      */
+static uint64_t nd_flat(uint64_t b, uint32_t e, const uint64_t d[3], const uint32_t be[3], const uint32_t ce[3]) {
+    uint64_t kz = ce[0] / be[0], ky = ce[1] / be[1], kx = ce[2] / be[2];
+    uint64_t bpc = kz * ky * kx;
+    uint64_t c = b / bpc, bi = b % bpc;
+    uint64_t gx = d[2] / ce[2], gy = d[1] / ce[1];
+    uint64_t cz = c / (gy * gx), cy = (c / gx) % gy, cx = c % gx;
+    uint64_t iz = bi / (ky * kx), iy = (bi / kx) % ky, ix = bi % kx;
+    uint64_t ez = e / (be[1] * be[2]), ey = (e / be[2]) % be[1], ex = e % be[2];
+    uint64_t z = cz * ce[0] + iz * be[0] + ez;
+    uint64_t y = cy * ce[1] + iy * be[1] + ey;
+    uint64_t x = cx * ce[2] + ix * be[2] + ex;
+    return (z * d[1] + y) * d[2] + x;
+}
+
+/* Lorenzo residuals of one block: q[] in block order -> d[] (as int32,
+ * modulo 2^32), neighbours outside the block are 0.                        */
+void orc_lorenzo_block(const int32_t *q, const uint32_t be[3], int32_t *d) {
+    for (uint32_t i = 0; i < be[0]; ++i)
+        for (uint32_t j = 0; j < be[1]; ++j)
+            for (uint32_t k = 0; k < be[2]; ++k) {
+                uint32_t acc = 0;
+                for (uint32_t a = 0; a < 2; ++a)
+                    for (uint32_t b = 0; b < 2; ++b)
+                        for (uint32_t c = 0; c < 2; ++c) {
+                            if (a > i || b > j || c > k) continue; /* outside the block: 0 */
+                            uint32_t v = (uint32_t)q[((i - a) * be[1] + (j - b)) * be[2] + (k - c)];
+                            acc = ((a + b + c) & 1u) ? acc - v : acc + v;
+                        }
+                d[(i * be[1] + j) * be[2] + k] = (int32_t)acc;
+            }
+}
+
+/* Inverse: inclusive prefix sums along x, then y, then z (modulo 2^32).    */
+void orc_unlorenzo_block(const int32_t *d, const uint32_t be[3], int32_t *q) {
+    uint32_t nb = be[0] * be[1] * be[2];
+    for (uint32_t e = 0; e < nb; ++e) q[e] = d[e];
+    for (uint32_t i = 0; i < be[0]; ++i)
+        for (uint32_t j = 0; j < be[1]; ++j)
+            for (uint32_t k = 1; k < be[2]; ++k) {
+                uint32_t e = (i * be[1] + j) * be[2] + k;
+                q[e] = (int32_t)((uint32_t)q[e] + (uint32_t)q[e - 1]);
+            }
+    for (uint32_t i = 0; i < be[0]; ++i)
+        for (uint32_t j = 1; j < be[1]; ++j)
+            for (uint32_t k = 0; k < be[2]; ++k) {
+                uint32_t e = (i * be[1] + j) * be[2] + k;
+                q[e] = (int32_t)((uint32_t)q[e] + (uint32_t)q[e - be[2]]);
+            }
+    for (uint32_t i = 1; i < be[0]; ++i)
+        for (uint32_t j = 0; j < be[1]; ++j)
+            for (uint32_t k = 0; k < be[2]; ++k) {
+                uint32_t e = (i * be[1] + j) * be[2] + k;
+                q[e] = (int32_t)((uint32_t)q[e] + (uint32_t)q[e - be[1] * be[2]]);
+            }
+}
+
+/* Compress an array of dims {Z, Y, X} (rank 3) or {1, Y, X} (rank 2) with
+ * the multi-dimensional Lorenzo predictor.  Same steps and stream as
+ * orc_compress otherwise.  Returns the stream length or ORC_ERR_*.        */
+int64_t orc_compress_lorenzo(const float *x, int rank, const uint64_t dims[3], uint32_t block, int abs_mode,
+                             double bound, uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
+    uint32_t be[3], ce[3];
+    if (!orc_nd_edges(rank, block, be, ce) || !(bound >= 0.0) || !isfinite(bound)) return ORC_ERR_ARG;
+    if ((rank == 2 && dims[0] != 1) || dims[0] % ce[0] || dims[1] % ce[1] || dims[2] % ce[2]) return ORC_ERR_ARG;
+    if (dims[0] > ORC_MAX_N || dims[1] > ORC_MAX_N || dims[2] > ORC_MAX_N) return ORC_ERR_ARG;
+    uint64_t n = dims[0] * dims[1] * dims[2];
+    if (n > ORC_MAX_N) return ORC_ERR_ARG;
+    if (fegetround() != FE_TONEAREST) return ORC_ERR_ARG;
+
+    float vmin = 0.0f, vmax = 0.0f;
+    if (!abs_mode) orc_value_range(x, n, &vmin, &vmax);
+    double eb;
+    float inv2eb, step;
+    orc_resolve_bound(abs_mode, bound, vmin, vmax, &eb, &inv2eb, &step);
+
+    uint64_t nb = n / block, nc = n / ORC_CHUNK, bpc = ORC_CHUNK / block;
+    int32_t *q = (int32_t *)malloc((n ? n : 1) * sizeof(int32_t));
+    uint8_t *flag = (uint8_t *)malloc(n ? n : 1);
+    uint8_t *width = (uint8_t *)malloc(nb ? nb : 1);
+    if (!q || !flag || !width) {
+        free(q); free(flag); free(width);
+        return ORC_ERR_NOMEM;
+    }
+    orc_quantize(x, n, inv2eb, step, eb, q, flag);
+    uint64_t m = 0, W = 0;
+    for (uint64_t i = 0; i < n; ++i) m += flag[i];
+
+    int32_t qb[256], db[256];
+    uint32_t z[256], words[256];
+    for (uint64_t b = 0; b < nb; ++b) {  /* widths */
+        for (uint32_t e = 0; e < block; ++e) qb[e] = q[nd_flat(b, e, dims, be, ce)];
+        orc_lorenzo_block(qb, be, db);
+        for (uint32_t e = 0; e < block; ++e) z[e] = orc_zigzag(db[e]);
+        width[b] = (uint8_t)orc_block_width(z, block);
+        W += orc_block_words(width[b], block);
+    }
+    orc_layout L = layout_of(nb, nc, W, m);
+    int64_t status = (int64_t)L.total;
+    if (m > outlier_cap) status = ORC_ERR_OUTLIER_CAP;
+    else if (L.total > out_cap) status = ORC_ERR_CAPACITY;
+    if (status < 0) {
+        free(q); free(flag); free(width);
+        return status;
+    }
+    memset(out, 0, L.total);
+    put_u32(out + 0, ORC_MAGIC);
+    put_u16(out + 4, (uint16_t)ORC_VERSION);
+    put_u16(out + 6, (uint16_t)((abs_mode ? ORC_FLAG_ABS : 0u) | ORC_FLAG_LORENZO_ND));
+    put_u64(out + 8, n);
+    put_u32(out + 16, block);
+    put_u32(out + 20, ORC_CHUNK);
+    put_f64(out + 24, eb);
+    put_f32(out + 32, inv2eb);
+    put_f32(out + 36, step);
+    put_f32(out + 40, vmin);
+    put_f32(out + 44, vmax);
+    put_u64(out + 48, nb);
+    put_u64(out + 56, nc);
+    put_u64(out + 64, W);
+    put_u64(out + 72, m);
+    put_u64(out + 80, L.total);
+    put_f64(out + 88, bound);
+    put_u64(out + 96, dims[0]);
+    put_u64(out + 104, dims[1]);
+    put_u64(out + 112, dims[2]);
+    memcpy(out + L.width_off, width, nb);
+
+    uint64_t rec = 0, before = 0;
+    for (uint64_t c = 0; c < nc; ++c) {
+        put_u32(out + L.index_off + 8 * c, (uint32_t)rec);
+        put_u32(out + L.index_off + 8 * c + 4, (uint32_t)before);
+        for (uint64_t b = c * bpc; b < (c + 1) * bpc; ++b) {
+            for (uint32_t e = 0; e < block; ++e) qb[e] = q[nd_flat(b, e, dims, be, ce)];
+            orc_lorenzo_block(qb, be, db);
+            for (uint32_t e = 0; e < block; ++e) z[e] = orc_zigzag(db[e]);
+            orc_pack_block(z, block, width[b], words);
+            uint32_t nw = orc_block_words(width[b], block);
+            for (uint32_t k = 0; k < nw; ++k) put_u32(out + L.record_off + 4 * (rec + k), words[k]);
+            rec += nw;
+        }
+        /* the brick's outliers, ascending C-order index: z, then y, then x */
+        uint64_t gx = dims[2] / ce[2], gy = dims[1] / ce[1];
+        uint64_t z0 = c / (gy * gx) * ce[0], y0 = (c / gx) % gy * ce[1], x0 = c % gx * ce[2];
+        uint64_t mc = 0, k = 0;
+        for (uint64_t zz = z0; zz < z0 + ce[0]; ++zz)
+            for (uint64_t yy = y0; yy < y0 + ce[1]; ++yy)
+                for (uint64_t xx = x0; xx < x0 + ce[2]; ++xx) mc += flag[(zz * dims[1] + yy) * dims[2] + xx];
+        for (uint64_t zz = z0; zz < z0 + ce[0]; ++zz)
+            for (uint64_t yy = y0; yy < y0 + ce[1]; ++yy)
+                for (uint64_t xx = x0; xx < x0 + ce[2]; ++xx) {
+                    uint64_t i = (zz * dims[1] + yy) * dims[2] + xx;
+                    if (!flag[i]) continue;
+                    uint32_t bits;
+                    memcpy(&bits, &x[i], 4);
+                    put_u32(out + L.record_off + 4 * (rec + k), (uint32_t)i);
+                    put_u32(out + L.record_off + 4 * (rec + mc + k), bits);
+                    ++k;
+                }
+        rec = rec + 2 * mc;   /* the brick's outlier indices and values */
+        before = before + mc;
+    }
+    free(q); free(flag); free(width);
+    return (int64_t)L.total;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Parsed header, exposed for the tests.                                     */
 typedef struct {
@@ -406,6 +636,7 @@ typedef struct {
     double eb, bound;
     float inv2eb, step, vmin, vmax;
     uint64_t width_off, index_off, record_off;
+    uint64_t dims[3];  /* Z, Y, X of a multi-dimensional Lorenzo stream, else 0 */
 } orc_header;
 
 int orc_parse_header(const uint8_t *s, uint64_t bytes, orc_header *h) {
@@ -428,9 +659,21 @@ int orc_parse_header(const uint8_t *s, uint64_t bytes, orc_header *h) {
     h->m = get_u64(s + 72);
     h->total = get_u64(s + 80);
     h->bound = get_f64(s + 88);
+    h->dims[0] = get_u64(s + 96);
+    h->dims[1] = get_u64(s + 104);
+    h->dims[2] = get_u64(s + 112);
     if (h->magic != ORC_MAGIC || h->version != ORC_VERSION || !block_ok(h->block) ||
         h->chunk != ORC_CHUNK)
         return ORC_ERR_CORRUPT;
+    if (h->flags & ORC_FLAG_LORENZO_ND) {
+        uint32_t be[3], ce[3];
+        int rank = h->dims[0] == 1 ? 2 : 3;
+        if (!orc_nd_edges(rank, h->block, be, ce) || h->dims[0] * h->dims[1] * h->dims[2] != h->n ||
+            h->dims[0] % ce[0] || h->dims[1] % ce[1] || h->dims[2] % ce[2])
+            return ORC_ERR_CORRUPT;
+    } else if (h->dims[0] || h->dims[1] || h->dims[2]) {
+        return ORC_ERR_CORRUPT;
+    }
     if (h->n > ORC_MAX_N || h->nb != (h->n + h->block - 1) / h->block ||
         h->nc != (h->n + ORC_CHUNK - 1) / ORC_CHUNK || h->W > h->n || h->m > h->n)
         return ORC_ERR_CORRUPT;
@@ -445,11 +688,14 @@ int orc_parse_header(const uint8_t *s, uint64_t bytes, orc_header *h) {
 /* Inverse ([SPEC] Inverse declaration; device policy contract: decode ->
  * undelta -> dequant code * 2eb), then each chunk's outliers are written
  * back over the reconstruction.                                            */
+static int decompress_nd(const uint8_t *s, const orc_header *h, float *out);
+
 int orc_decompress(const uint8_t *s, uint64_t bytes, float *out, uint64_t n_expected) {
     orc_header h;
     int rc = orc_parse_header(s, bytes, &h);
     if (rc != 0) return rc;
     if (h.n != n_expected) return ORC_ERR_ARG;
+    if (h.flags & ORC_FLAG_LORENZO_ND) return decompress_nd(s, &h, out);
 
     uint32_t words[256], z[256];
     uint64_t blocks_per_chunk = ORC_CHUNK / h.block;
@@ -493,6 +739,54 @@ int orc_decompress(const uint8_t *s, uint64_t bytes, float *out, uint64_t n_expe
         }
     }
     if (W_seen != h.W) return ORC_ERR_CORRUPT;
+    return 0;
+}
+
+/* Inverse of orc_compress_lorenzo: per brick, each block's codes unpacked,
+ * the Lorenzo residuals summed back (inclusive prefix sums along x, y, z
+ * within the block), dequantized and placed at their C-order positions;
+ * then the brick's outliers written back.                                  */
+static int decompress_nd(const uint8_t *s, const orc_header *h, float *out) {
+    uint32_t be[3], ce[3];
+    int rank = h->dims[0] == 1 ? 2 : 3;
+    if (!orc_nd_edges(rank, h->block, be, ce)) return ORC_ERR_CORRUPT;
+    uint32_t words[256], z[256];
+    int32_t d[256], q[256];
+    uint64_t bpc = ORC_CHUNK / h->block, R = h->W + 2 * h->m, W_seen = 0;
+    uint64_t gx = h->dims[2] / ce[2], gy = h->dims[1] / ce[1];
+    for (uint64_t c = 0; c < h->nc; ++c) {
+        uint64_t rec = get_u32(s + h->index_off + 8 * c);
+        uint64_t before = get_u32(s + h->index_off + 8 * c + 4);
+        uint64_t rec_next = (c + 1 < h->nc) ? get_u32(s + h->index_off + 8 * (c + 1)) : R;
+        uint64_t after = (c + 1 < h->nc) ? get_u32(s + h->index_off + 8 * (c + 1) + 4) : h->m;
+        if (rec_next < rec || after < before || rec_next > R || after > h->m) return ORC_ERR_CORRUPT;
+        uint64_t mc = after - before, word_off = rec;
+        for (uint64_t b = c * bpc; b < (c + 1) * bpc; ++b) {
+            uint32_t w = s[h->width_off + b];
+            if (w > 32) return ORC_ERR_CORRUPT;
+            uint32_t nw = orc_block_words(w, h->block);
+            if (word_off + nw > rec_next) return ORC_ERR_CORRUPT;
+            for (uint32_t k = 0; k < nw; ++k) words[k] = get_u32(s + h->record_off + 4 * (word_off + k));
+            orc_unpack_block(words, h->block, w, z);
+            for (uint32_t e = 0; e < h->block; ++e) d[e] = orc_unzigzag(z[e]);
+            orc_unlorenzo_block(d, be, q);
+            for (uint32_t e = 0; e < h->block; ++e) out[nd_flat(b, e, h->dims, be, ce)] = dequant(q[e], h->step);
+            word_off += nw;
+        }
+        if (word_off + 2 * mc != rec_next) return ORC_ERR_CORRUPT;
+        W_seen += word_off - rec;
+        uint64_t z0 = c / (gy * gx) * ce[0], y0 = (c / gx) % gy * ce[1], x0 = c % gx * ce[2];
+        for (uint64_t k = 0; k < mc; ++k) {
+            uint32_t i = get_u32(s + h->record_off + 4 * (word_off + k));
+            uint32_t bits = get_u32(s + h->record_off + 4 * (word_off + mc + k));
+            uint64_t xx = i % h->dims[2], yy = (i / h->dims[2]) % h->dims[1], zz = i / (h->dims[2] * h->dims[1]);
+            if (i >= h->n || zz < z0 || zz >= z0 + ce[0] || yy < y0 || yy >= y0 + ce[1] || xx < x0 ||
+                xx >= x0 + ce[2])
+                return ORC_ERR_CORRUPT;
+            memcpy(&out[i], &bits, 4);
+        }
+    }
+    if (W_seen != h->W) return ORC_ERR_CORRUPT;
     return 0;
 }
 

@@ -29,12 +29,19 @@ MUTATIONS = [
     ("no canonical +0", "*vmin_out = lo + 0.0f;", "*vmin_out = lo;"),
     ("inverse zigzag", "return (int32_t)(-(int64_t)(z / 2u) - 1);", "return (int32_t)(-(int64_t)(z / 2u));"),
     ("dequantisation", "return (float)q * step; }", "return (float)q * step * 1.0000001f; }"),
+    ("given range ignored", "if (!abs_mode && range) {", "if (!abs_mode && range && 0) {"),
+    ("Lorenzo stencil corner sign", "acc = ((a + b + c) & 1u) ? acc - v : acc + v;",
+     "acc = ((a + b) & 1u) ? acc - v : acc + v;"),
+    ("Lorenzo inverse along y", "q[e] = (int32_t)((uint32_t)q[e] + (uint32_t)q[e - be[2]]);",
+     "q[e] = (int32_t)((uint32_t)q[e] + (uint32_t)q[e - 1]);"),
+    ("block z index", "uint64_t z = cz * ce[0] + iz * be[0] + ez;", "uint64_t z = cz * ce[0] + iz * be[0];"),
 ]
 
 
 def _run_pins(src_path: str) -> subprocess.CompletedProcess:
     env = dict(os.environ, EBLC_ORACLE_SRC=src_path, PYTHONDONTWRITEBYTECODE="1")
     return subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_oracle_pins.py"),
+                           os.path.join(ROOT, "tests", "test_oracle_nd_pins.py"),
                            "-x", "-q", "-p", "no:cacheprovider", "-k", "not fuzz"],
                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
 

@@ -482,3 +482,70 @@ def test_stream_invariants_fuzz_multichunk(orc):
         _check_stream(orc, x, s, block)
 
     check()
+
+
+# ---------------------------------------------------------------------------
+# compress_range: one part of a larger array under the whole array's bound.
+
+def _chunk_records(s):
+    """Per chunk: (width bytes of its blocks, its record words) of a stream."""
+    P = SC.parts(s)
+    h = P["h"]
+    rec = P["raw"][P["off"]["record"]:P["off"]["total"]].view(np.uint32)
+    R = h["W"] + 2 * h["m"]
+    starts = list(P["index"][:, 0]) + [R]
+    bpc = SC.CHUNK // h["block"]
+    return [(P["widths"][c * bpc:(c + 1) * bpc].copy(), rec[starts[c]:starts[c + 1]].copy())
+            for c in range(h["nc"])]
+
+
+@pytest.mark.parametrize("block", BLOCKS)
+def test_compress_range_with_own_range_is_compress(orc, block):
+    for x in (WL.with_spikes((12, 32, 48), 2, p_nonfinite=1e-3), WL.edge_mix(9001, block), WL.sine_noise(5000, 1)):
+        lo, hi, _ = orc.value_range(x)
+        assert np.array_equal(orc.compress_range(x, block, 1e-3, lo, hi), orc.compress(x, block, rel=1e-3))
+
+
+@pytest.mark.parametrize("block", BLOCKS)
+@pytest.mark.parametrize("parts", [2, 3, 5])
+def test_compress_range_shards_match_the_whole_stream(orc, block, parts):
+    """Chunk-aligned parts coded under the whole array's range: each part's
+    stream passes every independent stream check with eb = rel * (vmax - vmin)
+    of the whole (exact rationals), and its width bytes, payload words and
+    outlier values are byte for byte those of the whole array's stream for
+    the same chunks (outlier indices count from the part's first element)."""
+    rel = 1e-3
+    x = np.concatenate([WL.kfield((8, 32, 64), 3), WL.with_spikes((8, 16, 64), 4, p_nonfinite=2e-3),
+                        WL.edge_mix(3 * 4096 + 77, 5)])
+    lo, hi, _ = orc.value_range(x)
+    eb = float(Fraction(rel) * Fraction(float(Fraction(float(np.float32(hi))) - Fraction(float(np.float32(lo))))))
+    whole = _chunk_records(orc.compress(x, block, rel=rel))
+    nc = -(-x.size // SC.CHUNK)
+    cuts = [0] + [(nc * k // parts) * SC.CHUNK for k in range(1, parts)] + [x.size]
+    c0 = 0
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        s = orc.compress_range(x[a:b], block, rel, lo, hi)
+        h = _check_stream(orc, x[a:b], s, block, eb_expected=eb)
+        assert h["vmin"] == np.float32(lo) and h["vmax"] == np.float32(hi) and h["flags"] == 0
+        mine = _chunk_records(s)
+        for k, (w, r) in enumerate(mine):
+            W, Rw = whole[c0 + k]
+            assert np.array_equal(w, W[:w.size]) and not W[w.size:].any()
+            # same payload words and outlier values; outlier indices are the
+            # part's own (element index within the part)
+            pw = int((-(-(w.astype(np.int64) * SC.block_counts(b - a, block)[
+                k * (SC.CHUNK // block):(k + 1) * (SC.CHUNK // block)]) // 32)).sum())
+            mc = (r.size - pw) // 2
+            assert r.size == Rw.size and pw + 2 * mc == r.size
+            assert np.array_equal(r[:pw], Rw[:pw]), (a, k)
+            assert np.array_equal(r[pw:pw + mc].astype(np.int64) + a, Rw[pw:pw + mc].astype(np.int64)), (a, k)
+            assert np.array_equal(r[pw + mc:], Rw[pw + mc:]), (a, k)
+        c0 += len(mine)
+    assert c0 == nc
+
+
+def test_compress_range_rejects_bad_ranges(orc):
+    x = WL.edge_mix(100, 1)
+    for lo, hi in ((1.0, 0.0), (np.nan, 1.0), (0.0, np.inf)):
+        with pytest.raises(orc.OracleError):
+            orc.compress_range(x, 64, 1e-3, lo, hi)
