@@ -18,10 +18,11 @@ constexpr uint32_t kHeaderBytes = 128;
 constexpr uint32_t kMagic = 0x434C4245u;  // "EBLC"
 constexpr uint32_t kVersion = 1;
 constexpr uint16_t kFlagAbs = 1;
+constexpr uint16_t kFlagLorenzoNd = 2;  // 2-D / 3-D Lorenzo over the array's dims (bytes 96..119: Z, Y, X)
 constexpr uint64_t kMaxN = 1ull << 30;
 
 // Device error word bits.
-enum : uint32_t { kErrTimeout = 1u, kErrCapacity = 2u, kErrCorrupt = 4u };
+enum : uint32_t { kErrTimeout = 1u, kErrCapacity = 2u, kErrCorrupt = 4u, kErrRange = 8u };
 
 __host__ __device__ constexpr uint64_t pad16(uint64_t v) { return (v + 15u) & ~uint64_t(15); }
 
@@ -46,6 +47,7 @@ struct Bound {
     float inv2eb, step;
     float t_in, t_out;  // |x - x'| (fp32) <= t_in: certainly within eb; > t_out: certainly not
     float vmin, vmax;
+    int check_range;    // 0: every finite element is known to give |x * inv2eb| < 2^30
 };
 
 // eb = rel * (vmax - vmin) (or the absolute bound), inv2eb = (float)(1/(2 eb)),
@@ -60,7 +62,7 @@ struct Bound {
 // more than one double ulp, so the fp64 test agrees in both cases.  Anything
 // in between (and NaN) takes the fp64 test.  For eb outside [2^-120, 1e37]
 // the filter is disabled (t_in = 0, t_out = inf).
-__device__ inline Bound resolve_bound(int abs_mode, double bound, float vmin, float vmax) {
+__device__ inline Bound resolve_bound(int abs_mode, double bound, float vmin, float vmax, int range_given = 0) {
     Bound b;
     b.vmin = abs_mode ? 0.0f : vmin;
     b.vmax = abs_mode ? 0.0f : vmax;
@@ -77,6 +79,14 @@ __device__ inline Bound resolve_bound(int abs_mode, double bound, float vmin, fl
         b.t_in = 0.0f;
         b.t_out = __int_as_float(0x7f800000);
     }
+    // Relative bound over the array's own range: every finite element lies in
+    // [vmin, vmax], and float rounding is monotone, so |fl(x * inv2eb)| <=
+    // fl(max(|vmin|, |vmax|) * inv2eb).  When that is below 2^30 the
+    // quantizer's range test can never fail for a finite element (non-finite
+    // ones fail the bound test anyway).  A range given by the caller is not
+    // trusted to contain the elements: the test stays on.
+    const float amax = fmaxf(fabsf(b.vmin), fabsf(b.vmax));
+    b.check_range = (abs_mode || range_given) ? 1 : !(__fmul_rn(amax, b.inv2eb) < 0x1p30f);
     return b;
 }
 
@@ -150,6 +160,69 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
         : "memory");
 }
 
+// Bulk prefetch of [src, src + bytes) into L2 (no completion, no shared
+// memory): puts more DRAM reads in flight than the shared-memory stages can
+// hold.  src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// 16-byte asynchronous copy global -> shared through L1 (cp.async), and the
+// arrive-on of an mbarrier once all of this thread's earlier cp.async have
+// landed (the mbarrier's expected count includes these arrivals).
+__device__ __forceinline__ void async_copy16(void *dst_smem, const void *src_gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
+}
+
+__device__ __forceinline__ void async_copy_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Tiled tensor copies global -> shared (one box of the tensor map at the
+// given element coordinates, x innermost) completing on an mbarrier, and
+// their L2 prefetch form.  The x coordinate times 4 bytes is a multiple of
+// 16 at every call site (bricks start at multiples of 16 elements).  Never
+// used with .multicast.
+__device__ __forceinline__ void tensor_g2s_3d(void *dst_smem, const void *tmap, int x, int y, int z, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(smem_u32(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tensor_g2s_2d(void *dst_smem, const void *tmap, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst_smem)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tensor_prefetch_3d(const void *tmap, int x, int y, int z) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tensor_prefetch_2d(const void *tmap, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
+
+// Brick t of a multi-dimensional array {Z, Y, X} in C order over the brick
+// grid: its first element's (z, y, x).
+__host__ __device__ inline void brick_origin(uint64_t t, int nd, const uint64_t *dims, int &z, int &y, int &x) {
+    const uint64_t ex = (nd == 3) ? 16 : 64, ey = ex, ez = (nd == 3) ? 16 : 1;
+    const uint64_t gx = dims[2] / ex, gy = dims[1] / ey;
+    x = (int)((t % gx) * ex);
+    y = (int)(((t / gx) % gy) * ey);
+    z = (int)((t / (gx * gy)) * ez);
+}
+
 __device__ __forceinline__ uint64_t ld_relaxed_gpu(const uint64_t *p) {
     uint64_t v;
     asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
@@ -158,11 +231,6 @@ __device__ __forceinline__ uint64_t ld_relaxed_gpu(const uint64_t *p) {
 
 __device__ __forceinline__ void st_relaxed_gpu(uint64_t *p, uint64_t v) {
     asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-// Named barrier among the first `threads` threads of the CTA (id 1..15).
-__device__ __forceinline__ void named_bar(uint32_t id, uint32_t threads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // Streaming store (written once, not re-read by this kernel).

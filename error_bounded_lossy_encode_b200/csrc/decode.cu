@@ -36,6 +36,10 @@ constexpr int kThreads = (kNW + 1) * 32;
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kStagedOutliers = 1024;                 // outliers staged with the payload
 constexpr uint32_t kRecWords = kChunk + 2 * kStagedOutliers + 4 + 16;  // + alignment + over-read slack
+#ifndef EBLC_DEC_PREFETCH
+#define EBLC_DEC_PREFETCH 0
+#endif
+constexpr int kPrefetch = EBLC_DEC_PREFETCH;  // chunks of this CTA whose records are fetched into L2 ahead
 
 struct __align__(128) DecSmem {
     uint32_t rec[kS][kRecWords];
@@ -57,12 +61,148 @@ __device__ __forceinline__ uint32_t group_scan_excl(uint32_t v, int r, uint32_t 
     return incl - v;
 }
 
-template <int V, int LPB>
+// Width of this lane's block and the exclusive prefix / total of the widths
+// of the warp-tile's blocks (wb: their width bytes in shared memory), read as
+// one word per lane instead of a shuffle per block.  Widths above 32 exist
+// only in corrupt streams: they are clamped to 32 (per byte, so the byte
+// sums below stay under 256) and reported through `raw_over`.
+template <int LPB>
+__device__ __forceinline__ void widths_of_tile(const uint8_t *wb, int g, uint32_t &w, uint32_t &pre, uint32_t &tot,
+                                               bool &raw_over) {
+    if constexpr (LPB == 32) {
+        const uint32_t raw = wb[0];
+        raw_over = raw > 32u;
+        w = min(raw, 32u);
+        pre = 0;
+        tot = w;
+    } else if constexpr (LPB == 16) {
+        const uint32_t raw = *reinterpret_cast<const uint16_t *>(wb);
+        const uint32_t c = __vminu4(raw, 0x2020u);
+        raw_over = ((raw >> (8 * g)) & 0xffu) > 32u;
+        const uint32_t w0 = c & 0xffu, w1 = c >> 8;
+        w = g ? w1 : w0;
+        pre = g ? w0 : 0u;
+        tot = w0 + w1;
+    } else if constexpr (LPB == 8) {
+        const uint32_t raw = *reinterpret_cast<const uint32_t *>(wb);
+        const uint32_t c = __vminu4(raw, 0x20202020u);
+        raw_over = ((raw >> (8 * g)) & 0xffu) > 32u;
+        w = (c >> (8 * g)) & 0xffu;
+        pre = ((c * 0x01010100u) >> (8 * g)) & 0xffu;
+        tot = (c * 0x01010101u) >> 24;
+    } else {  // LPB == 4: eight blocks in two words
+        const uint2 raw = *reinterpret_cast<const uint2 *>(wb);
+        const uint32_t lo = __vminu4(raw.x, 0x20202020u), hi = __vminu4(raw.y, 0x20202020u);
+        const uint32_t rw = (g < 4) ? raw.x : raw.y, cw = (g < 4) ? lo : hi;
+        raw_over = ((rw >> (8 * (g & 3))) & 0xffu) > 32u;
+        const uint32_t tlo = (lo * 0x01010101u) >> 24;
+        w = (cw >> (8 * (g & 3))) & 0xffu;
+        pre = ((cw * 0x01010100u) >> (8 * (g & 3))) & 0xffu;
+        if (g >= 4) pre += tlo;
+        tot = tlo + ((hi * 0x01010101u) >> 24);
+    }
+}
+
+// Multi-dimensional Lorenzo blocks (nd = 2, 3): the lane's residuals d (8
+// codes in block order, the encoder's lane layout: 3-D 4x4x4 two rows of 4;
+// 3-D 4x8x8 and 2-D 8x8 one row of 8; 2-D 16x16 half a row) summed back --
+// inclusive prefix sums along x, then y, then z within the block, by
+// segmented warp scans -- dequantized and stored at their places in the
+// array.  Brick t's block bi (C order within the brick).
+template <int ND, int LPB>
+__device__ __forceinline__ void nd_store(const DecodeArgs &a, int tile, uint32_t bi, int r, const uint32_t (&d)[8]) {
+    constexpr int kBX = (ND == 3) ? (LPB == 8 ? 4 : 8) : (LPB == 8 ? 8 : 16);
+    constexpr int kBY = (ND == 3) ? (LPB == 8 ? 4 : 8) : (LPB == 8 ? 8 : 16);
+    constexpr int kKX = ((ND == 3) ? 16 : 64) / kBX, kKY = ((ND == 3) ? 16 : 64) / kBY;
+    uint32_t q[8];
+    int zo, yo, xo;  // the lane's first code, within the block
+    if constexpr (ND == 3 && LPB == 8) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) q[v] = d[v] + ((v & 3) ? q[v - 1] : 0u);  // x, per row of 4
+#pragma unroll
+        for (int v = 0; v < 4; ++v) q[v + 4] += q[v];                            // y, within the lane
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {                                             // y, rows 0-1 of lane r-1
+            const uint32_t up = __shfl_up_sync(kFull, q[v + 4], 1);
+            if (r & 1) { q[v] += up; q[v + 4] += up; }
+        }
+#pragma unroll
+        for (int o = 2; o <= 4; o <<= 1)                                         // z: planes at lane stride 2
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const uint32_t up = __shfl_up_sync(kFull, q[v], o);
+                if (r >= o) q[v] += up;
+            }
+        zo = r >> 1; yo = (r & 1) << 1; xo = 0;
+    } else if constexpr (ND == 3) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) q[v] = d[v] + (v ? q[v - 1] : 0u);
+#pragma unroll
+        for (int o = 1; o <= 4; o <<= 1)                                         // y: rows at lane stride 1
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const uint32_t up = __shfl_up_sync(kFull, q[v], o);
+                if ((r & 7) >= o) q[v] += up;
+            }
+#pragma unroll
+        for (int o = 8; o <= 16; o <<= 1)                                        // z: planes at lane stride 8
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const uint32_t up = __shfl_up_sync(kFull, q[v], o);
+                if (r >= o) q[v] += up;
+            }
+        zo = r >> 3; yo = r & 7; xo = 0;
+    } else if constexpr (LPB == 8) {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) q[v] = d[v] + (v ? q[v - 1] : 0u);
+#pragma unroll
+        for (int o = 1; o <= 4; o <<= 1)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const uint32_t up = __shfl_up_sync(kFull, q[v], o);
+                if (r >= o) q[v] += up;
+            }
+        zo = 0; yo = r; xo = 0;
+    } else {
+#pragma unroll
+        for (int v = 0; v < 8; ++v) q[v] = d[v] + (v ? q[v - 1] : 0u);
+        const uint32_t left = __shfl_up_sync(kFull, q[7], 1);                    // x: first half of the row
+        if (r & 1) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) q[v] += left;
+        }
+#pragma unroll
+        for (int o = 2; o <= 16; o <<= 1)                                        // y: rows at lane stride 2
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                const uint32_t up = __shfl_up_sync(kFull, q[v], o);
+                if (r >= o) q[v] += up;
+            }
+        zo = 0; yo = r >> 1; xo = (r & 1) << 3;
+    }
+    float y[8];
+#pragma unroll
+    for (int v = 0; v < 8; ++v) y[v] = __fmul_rn(__int2float_rn((int32_t)q[v]), a.step);
+    int bz, by, bx;
+    brick_origin((uint64_t)tile, ND, a.dims, bz, by, bx);
+    const int kx = (int)(bi % kKX), ky = (int)((bi / kKX) % kKY), kz = (int)(bi / (kKX * kKY));
+    const uint64_t z = (uint64_t)(bz + kz * ((ND == 3) ? 4 : 1) + zo);
+    const uint64_t yy = (uint64_t)(by + ky * kBY + yo), x = (uint64_t)(bx + kx * kBX + xo);
+    float *row = a.out + (z * a.dims[1] + yy) * a.dims[2] + x;
+    if constexpr (ND == 3 && LPB == 8) {  // two rows of 4
+        __stcs(reinterpret_cast<float4 *>(row), make_float4(y[0], y[1], y[2], y[3]));
+        __stcs(reinterpret_cast<float4 *>(row + a.dims[2]), make_float4(y[4], y[5], y[6], y[7]));
+    } else {
+        __stcs(reinterpret_cast<float4 *>(row), make_float4(y[0], y[1], y[2], y[3]));
+        __stcs(reinterpret_cast<float4 *>(row + 4), make_float4(y[4], y[5], y[6], y[7]));
+    }
+}
+
+template <int V, int LPB, int ND>
 __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
     constexpr int kB = V * LPB;
     constexpr int kWT = 32 * V;
     constexpr int kWPW = kChunk / kWT / kNW;
-    constexpr int kGroups = 32 / LPB;
     constexpr int kEPL = kB / 32;  // payload words per unit of width for a full block
     const int g = ln / LPB, r = ln % LPB;
     const int tid = cw * 32 + ln;
@@ -91,33 +231,64 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
                 const int wt = cw * kWPW + k;
                 const uint32_t e0 = wt * kWT + ln * V;
                 const uint32_t blk = (uint32_t)(wt * kWT) / kB + g;
-                uint32_t w = wid[blk];
-                if (w > 32u) {
-                    if (r == 0 && blk * kB < valid) atomicOr(a.err, kErrCorrupt);
-                    w = 32u;
-                }
-                uint32_t pre = 0, tot = 0;
-#pragma unroll
-                for (int gg = 0; gg < kGroups; ++gg) {
-                    const uint32_t b = __shfl_sync(kFull, w, gg * LPB);
-                    pre += (gg < g) ? b : 0u;
-                    tot += b;
-                }
+                uint32_t w, pre, tot;
+                bool over;
+                widths_of_tile<LPB>(wid + (uint32_t)(wt * kWT) / kB, g, w, pre, tot, over);
+                if (over && r == 0 && blk * kB < valid) atomicOr(a.err, kErrCorrupt);
                 // bit position of this lane's first code in the chunk payload
                 const uint32_t bit0 = 32u * kEPL * (before + pre) + (uint32_t)r * V * w;
                 const uint32_t mask = (w == 32u) ? kFull : ((1u << w) - 1u);
                 int32_t c[V];
+                uint32_t dv[V];  // the residuals (the 1-D path also keeps their running sum in c)
                 uint32_t run = 0;
-                // Every word this lane reads lies in the staged record (widths
-                // checked above): one test for the lane instead of one per code.
+                // The lane's codes occupy bits [bit0, bit0 + 8w) of the staged
+                // payload.  For narrow blocks the lane loads the few words that
+                // hold them once and shifts the codes out of registers; wider
+                // blocks read two words per code.  Every word read lies in the
+                // staged record (widths checked above): one test per lane.
+                const uint32_t wmax = __reduce_max_sync(kFull, w);
+                const uint32_t wd0 = bit0 >> 5, sh0 = bit0 & 31u;
                 const bool inside = ((bit0 + V * w) >> 5) + 1 < kRecWords - adj;
-                if (__all_sync(kFull, inside)) {
+                if (wmax <= 8u && __all_sync(kFull, wd0 + 2 < kRecWords - adj)) {
+                    static_assert(V == 8, "narrow path: 8 codes of <= 8 bits fit in 64 bits");
+                    uint32_t lo = __funnelshift_r(rec[wd0], rec[wd0 + 1], sh0);
+                    uint32_t hi = __funnelshift_r(rec[wd0 + 1], rec[wd0 + 2], sh0);
+#pragma unroll
+                    for (int v = 0; v < V; ++v) {
+                        const uint32_t zz = lo & mask;
+                        lo = __funnelshift_r(lo, hi, w);
+                        hi >>= w;
+                        const uint32_t d = (zz >> 1) ^ (0u - (zz & 1u));  // inverse zigzag
+                        dv[v] = d;
+                        run += d;
+                        c[v] = (int32_t)run;
+                    }
+                } else if (wmax <= 16u && __all_sync(kFull, wd0 + 4 < kRecWords - adj)) {
+                    // 8 codes of <= 16 bits: 128 bits, shifted out of four words
+                    uint32_t g0 = __funnelshift_r(rec[wd0], rec[wd0 + 1], sh0);
+                    uint32_t g1 = __funnelshift_r(rec[wd0 + 1], rec[wd0 + 2], sh0);
+                    uint32_t g2 = __funnelshift_r(rec[wd0 + 2], rec[wd0 + 3], sh0);
+                    uint32_t g3 = __funnelshift_r(rec[wd0 + 3], rec[wd0 + 4], sh0);
+#pragma unroll
+                    for (int v = 0; v < V; ++v) {
+                        const uint32_t zz = g0 & mask;
+                        g0 = __funnelshift_r(g0, g1, w);
+                        g1 = __funnelshift_r(g1, g2, w);
+                        g2 = __funnelshift_r(g2, g3, w);
+                        g3 >>= w;
+                        const uint32_t d = (zz >> 1) ^ (0u - (zz & 1u));  // inverse zigzag
+                        dv[v] = d;
+                        run += d;
+                        c[v] = (int32_t)run;
+                    }
+                } else if (__all_sync(kFull, inside)) {
 #pragma unroll
                     for (int v = 0; v < V; ++v) {
                         const uint32_t b = bit0 + v * w;
                         const uint32_t wd = b >> 5;
                         const uint32_t zz = __funnelshift_r(rec[wd], rec[wd + 1], b & 31u) & mask;
                         const uint32_t d = (zz >> 1) ^ (0u - (zz & 1u));  // inverse zigzag
+                        dv[v] = d;
                         run += d;
                         c[v] = (int32_t)run;
                     }
@@ -130,9 +301,15 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
                                                 ? (__funnelshift_r(rec[wd], rec[wd + 1], b & 31u) & mask)
                                                 : 0u;
                         const uint32_t d = (zz >> 1) ^ (0u - (zz & 1u));  // inverse zigzag
+                        dv[v] = d;
                         run += d;
                         c[v] = (int32_t)run;
                     }
+                }
+                if constexpr (ND != 0) {
+                    nd_store<ND, LPB>(a, tile, (uint32_t)(wt * kWT) / kB + g, r, dv);
+                    before += tot;
+                    continue;
                 }
                 uint32_t incl;
                 const uint32_t ex = group_scan_excl<LPB>(run, r, incl);
@@ -180,11 +357,24 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
             for (uint32_t k = tid; k < mt; k += kNW * 32) {
                 const uint32_t idx = staged ? rec[PW + k] : gidx[k];
                 const uint32_t val = staged ? rec[PW + mt + k] : gidx[mt + k];
-                const uint64_t e = (uint64_t)idx - (uint64_t)tile * kChunk;
-                if (idx >= (uint64_t)tile * kChunk && e < valid)
-                    gout[e] = __uint_as_float(val);
-                else
-                    atomicOr(a.err, kErrCorrupt);
+                if constexpr (ND != 0) {  // the index must lie in this brick
+                    int bz, by, bx;
+                    brick_origin((uint64_t)tile, ND, a.dims, bz, by, bx);
+                    const uint64_t xx = idx % a.dims[2], yy = (idx / a.dims[2]) % a.dims[1];
+                    const uint64_t zz = idx / (a.dims[2] * a.dims[1]);
+                    const uint64_t ez = (ND == 3) ? 16 : 1, exy = (ND == 3) ? 16 : 64;
+                    if (idx < a.n && zz >= (uint64_t)bz && zz < bz + ez && yy >= (uint64_t)by && yy < by + exy &&
+                        xx >= (uint64_t)bx && xx < bx + exy)
+                        a.out[idx] = __uint_as_float(val);
+                    else
+                        atomicOr(a.err, kErrCorrupt);
+                } else {
+                    const uint64_t e = (uint64_t)idx - (uint64_t)tile * kChunk;
+                    if (idx >= (uint64_t)tile * kChunk && e < valid)
+                        gout[e] = __uint_as_float(val);
+                    else
+                        atomicOr(a.err, kErrCorrupt);
+                }
             }
         }
         __syncwarp();
@@ -198,10 +388,24 @@ __device__ void producer_warp(DecSmem &sm, const DecodeArgs &a, int ln) {
     const uint64_t R = a.W + 2 * a.m;
     const uint32_t K = kChunk / a.block;  // blocks per chunk
     const uint64_t total16 = a.total & ~uint64_t(15);
+    // L2 prefetch of the record of this CTA's chunk of iteration j (its
+    // extent from the chunk index, clamped to the stream; only a hint, so a
+    // corrupt index costs nothing but the prefetch).
+    auto prefetch_record = [&](uint32_t j) {
+        const uint64_t tp = (uint64_t)blockIdx.x + (uint64_t)j * gridDim.x;
+        if (tp >= L.nc) return;
+        const uint64_t r0 = *reinterpret_cast<const uint32_t *>(a.in + L.index_off + 8 * tp);
+        const uint64_t r1 = (tp + 1 < L.nc) ? *reinterpret_cast<const uint32_t *>(a.in + L.index_off + 8 * (tp + 1)) : R;
+        const uint64_t b0 = (L.record_off + 4 * r0) & ~uint64_t(15);
+        const uint64_t b1 = min((L.record_off + 4 * r1 + 15) & ~uint64_t(15), total16);
+        if (r1 > r0 && b1 > b0 && b1 - b0 <= 4ull * kRecWords) prefetch_l2(a.in + b0, (uint32_t)(b1 - b0));
+    };
+    for (uint32_t j = 1; j <= (uint32_t)kPrefetch; ++j) prefetch_record(j);
     uint32_t i = 0;
     for (;; ++i) {
         const int s = i % kS;
         if (i >= kS && !mbar_wait(&sm.empty[s], ((i / kS) - 1) & 1, a.wait_ns, a.err)) break;
+        if (i >= 1 && kPrefetch > 0) prefetch_record(i + kPrefetch);
         const uint64_t t = (uint64_t)blockIdx.x + (uint64_t)i * gridDim.x;
         if (t >= L.nc) {
             sm.info[s][0] = (uint32_t)-1;
@@ -266,7 +470,7 @@ __device__ void producer_warp(DecSmem &sm, const DecodeArgs &a, int ln) {
     }
 }
 
-template <int V, int LPB>
+template <int V, int LPB, int ND>
 __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeArgs a) {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     DecSmem &sm = *reinterpret_cast<DecSmem *>(smem_raw);
@@ -281,22 +485,22 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeArgs a)
     }
     __syncthreads();
     if (warp < kNW)
-        compute_warp<V, LPB>(sm, a, warp, ln);
+        compute_warp<V, LPB, ND>(sm, a, warp, ln);
     else
         producer_warp(sm, a, ln);
 }
 
-template <int V, int LPB>
+template <int V, int LPB, int ND>
 cudaError_t launch_t(const DecodeArgs &a, int num_sms, cudaStream_t stream) {
     const size_t smem = sizeof(DecSmem);
     cudaError_t e =
-        cudaFuncSetAttribute(decode_kernel<V, LPB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(decode_kernel<V, LPB, ND>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const uint64_t nc = (a.n + kChunk - 1) / kChunk;
     if (nc == 0) return cudaSuccess;
     const uint64_t want = (uint64_t)num_sms * 4;
     const int grid = (int)(want < nc ? want : nc);
-    decode_kernel<V, LPB><<<grid, kThreads, smem, stream>>>(a);
+    decode_kernel<V, LPB, ND><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -304,10 +508,14 @@ cudaError_t launch_t(const DecodeArgs &a, int num_sms, cudaStream_t stream) {
 
 cudaError_t launch_decode(const DecodeArgs &a, int num_sms, cudaStream_t stream) {
     switch (a.block) {
-        case 32: return launch_t<8, 4>(a, num_sms, stream);
-        case 64: return launch_t<8, 8>(a, num_sms, stream);
-        case 128: return launch_t<8, 16>(a, num_sms, stream);
-        case 256: return launch_t<8, 32>(a, num_sms, stream);
+        case 32: return a.nd ? cudaErrorInvalidValue : launch_t<8, 4, 0>(a, num_sms, stream);
+        case 64: return a.nd == 3 ? launch_t<8, 8, 3>(a, num_sms, stream)
+                      : a.nd == 2 ? launch_t<8, 8, 2>(a, num_sms, stream)
+                                  : launch_t<8, 8, 0>(a, num_sms, stream);
+        case 128: return a.nd ? cudaErrorInvalidValue : launch_t<8, 16, 0>(a, num_sms, stream);
+        case 256: return a.nd == 3 ? launch_t<8, 32, 3>(a, num_sms, stream)
+                       : a.nd == 2 ? launch_t<8, 32, 2>(a, num_sms, stream)
+                                   : launch_t<8, 32, 0>(a, num_sms, stream);
         default: return cudaErrorInvalidValue;
     }
 }

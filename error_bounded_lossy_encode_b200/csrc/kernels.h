@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>  // CUtensorMap (the tensor map itself is encoded on the host)
 #include <cuda_runtime.h>
 
 namespace eblc {
@@ -30,7 +31,8 @@ struct EncodeArgs {
     uint32_t block;           // 32, 64, 128, 256
     int abs_mode;
     double bound;             // relative or absolute bound as requested
-    const float *range;       // vmin, vmax from the range kernel (relative mode)
+    const float *range;       // vmin, vmax (relative mode): from the range kernel, or given by the caller
+    int range_given;          // 1: `range` comes from the caller (checked: finite, vmin <= vmax)
     uint64_t *status;         // look-back words: two arrays of ntiles; the call uses array
                               // (*epoch & 1), zero on entry, and clears the other one
     uint64_t ntiles;          // stride between the two arrays
@@ -40,6 +42,12 @@ struct EncodeArgs {
     uint64_t outlier_cap;
     int64_t stall_tile;       // test hook (-1: off)
     uint64_t wait_ns;         // limit of every device-side wait
+    // Multi-dimensional Lorenzo (nd = 2 or 3; 0: the 1-D path): the array's
+    // dims {Z, Y, X} (Z = 1 for 2-D), each a multiple of the brick edge, and
+    // a tiled tensor map of `in` with a 16x16x16 (3-D) or 64x64 (2-D) box.
+    int nd;
+    uint64_t dims[3];
+    CUtensorMap tmap;
 };
 cudaError_t launch_encode(const EncodeArgs &a, int num_sms, cudaStream_t stream);
 
@@ -71,6 +79,8 @@ struct DecodeArgs {
     float *out;               // n floats, 16-byte aligned
     uint32_t *err;            // sticky error word (kErrCorrupt, kErrTimeout)
     uint64_t wait_ns;
+    int nd;                   // as EncodeArgs::nd
+    uint64_t dims[3];         // {Z, Y, X} when nd != 0
 };
 cudaError_t launch_decode(const DecodeArgs &a, int num_sms, cudaStream_t stream);
 
