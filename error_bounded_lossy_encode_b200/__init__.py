@@ -11,6 +11,8 @@ Functions keep the C names::
     st, lim  = eblc_plan_get_limits(plan)
     st, nbytes = eblc_compress(plan, cuda_exec(stream), d_in, d_out, capacity, sidecar)
     st = eblc_compress_async(plan, cuda_exec(stream), d_in, d_out, capacity, d_result)   # no host sync
+    st = eblc_value_range(plan, cuda_exec(stream), d_in, d_range)                       # device float[2]
+    st, nbytes = eblc_compress_range(plan, cuda_exec(stream), d_in, d_range, d_out, capacity, sidecar)
     st = eblc_decompress(plan, cuda_exec(stream), d_stream, nbytes, sidecar, d_out)
     st = eblc_check(plan, cuda_exec(stream))
     eblc_plan_destroy(plan)
@@ -96,6 +98,11 @@ def lib() -> ctypes.CDLL:
     L.eblc_compress.restype = i32
     L.eblc_compress_async.argtypes = [P, ctypes.POINTER(eblc_execution_t), P, P, ctypes.c_size_t, P]
     L.eblc_compress_async.restype = i32
+    L.eblc_value_range.argtypes = [P, ctypes.POINTER(eblc_execution_t), P, P]
+    L.eblc_value_range.restype = i32
+    L.eblc_compress_range.argtypes = [P, ctypes.POINTER(eblc_execution_t), P, P, P, ctypes.c_size_t,
+                                      ctypes.POINTER(ctypes.c_size_t), P]
+    L.eblc_compress_range.restype = i32
     L.eblc_decompress.argtypes = [P, ctypes.POINTER(eblc_execution_t), P, ctypes.c_size_t, P, P]
     L.eblc_decompress.restype = i32
     L.eblc_check.argtypes = [P, ctypes.POINTER(eblc_execution_t)]
@@ -158,6 +165,23 @@ def eblc_compress_async(plan, exec_: eblc_execution_t, d_in: int, d_out: int, ou
     eblc_async_result_t (32 bytes) at d_result.  Returns the queueing status."""
     return lib().eblc_compress_async(plan, ctypes.byref(exec_), ctypes.c_void_p(d_in or None),
                                      ctypes.c_void_p(d_out or None), out_capacity, ctypes.c_void_p(d_result or None))
+
+
+def eblc_value_range(plan, exec_: eblc_execution_t, d_in: int, d_range: int) -> int:
+    """Queue the value range of d_in into the device float[2] at d_range."""
+    return lib().eblc_value_range(plan, ctypes.byref(exec_), ctypes.c_void_p(d_in or None),
+                                  ctypes.c_void_p(d_range or None))
+
+
+def eblc_compress_range(plan, exec_: eblc_execution_t, d_in: int, d_range: int, d_out: int, out_capacity: int,
+                        sidecar: eblc_sidecar_t | None = None):
+    """Compress under the value range in the device float[2] at d_range.
+    Returns (status, compressed_bytes)."""
+    nbytes = ctypes.c_size_t(0)
+    st = lib().eblc_compress_range(plan, ctypes.byref(exec_), ctypes.c_void_p(d_in or None),
+                                   ctypes.c_void_p(d_range or None), ctypes.c_void_p(d_out or None), out_capacity,
+                                   ctypes.byref(nbytes), None if sidecar is None else ctypes.byref(sidecar))
+    return st, int(nbytes.value)
 
 
 def async_result(raw) -> dict:

@@ -20,6 +20,8 @@
 #include <new>
 #include <string>
 
+#include <cudaTypedefs.h>  // PFN_cuTensorMapEncodeTiled
+
 #include "../../include/eblc.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -82,6 +84,8 @@ struct eblc_plan_s {
     uint64_t outlier_cap = 0;
     uint64_t wait_ns = 2000ull * 1000000ull;
     int64_t stall_tile = -1;
+    int nd = 0;                     // option lorenzo=nd: 2 or 3 (the plan's rank), 0 for the 1-D path
+    uint64_t dims[3] = {0, 0, 0};   // {Z, Y, X} of a multi-dimensional plan (Z = 1 for 2-D)
     uint64_t stall_call = 0;        // the compress call (0-based) that stall_tile applies to
     uint64_t calls = 0;             // compress calls enqueued so far
     Layout L{};
@@ -194,6 +198,9 @@ eblc_status_t parse_options(const char *options, eblc_plan_s *p, bool *timing) {
         } else if (key == "outlier_cap") {
             if (!parse_int(val, &iv) || iv < 0) return EBLC_INVALID_ARG;
             p->outlier_cap = (uint64_t)iv;  // clamped to n by the caller
+        } else if (key == "lorenzo") {
+            if (val == "nd") p->nd = -1;  // resolved against the dims by the caller
+            else if (val != "1d") return EBLC_INVALID_ARG;
         } else if (key == "timing") {
             if (!parse_int(val, &iv)) return EBLC_INVALID_ARG;
             *timing = iv != 0;
@@ -278,13 +285,45 @@ eblc_status_t ensure_host_staging(eblc_plan_s *p) {
 // the caller brackets a larger span, e.g. the HOST kind's copies).
 // d_user: NULL for the synchronous calls (the result block is copied to the
 // pinned readback), else the caller's device result record (no copy back).
+// Tiled tensor map of a multi-dimensional plan's input at d_in: dims {X, Y[, Z]}
+// innermost first, a brick (16^3, or 64x64 in 2-D) per box, no swizzle, so a
+// box lands in shared memory in C order.  The encoder is taken from the
+// driver once per process.
+eblc_status_t encode_tensor_map(const eblc_plan_s *p, const float *d_in, CUtensorMap *out) {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            f = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    if (!fn) return EBLC_CUDA_ERROR;
+    const cuuint32_t rank = (cuuint32_t)p->nd;
+    cuuint64_t gdim[3] = {p->dims[2], p->dims[1], p->dims[0]};
+    cuuint64_t gstride[2] = {p->dims[2] * 4, p->dims[2] * p->dims[1] * 4};  // bytes, of dims 1 and 2
+    cuuint32_t box[3] = {(p->nd == 3) ? 16u : 64u, (p->nd == 3) ? 16u : 64u, 16u};
+    cuuint32_t estride[3] = {1, 1, 1};
+    const CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank, const_cast<float *>(d_in), gdim, gstride, box,
+                          estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        EBLC_LOG("cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return EBLC_CUDA_ERROR;
+    }
+    return EBLC_OK;
+}
+
+// given_range: NULL, or a device float[2] {vmin, vmax} that replaces the
+// value range of d_in (relative bound; the range kernel is not run).
 eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_in, uint8_t *d_out, uint64_t cap,
-                               bool call_events = true, uint64_t *d_user = nullptr) {
+                               bool call_events = true, uint64_t *d_user = nullptr,
+                               const float *given_range = nullptr) {
     if (call_events)
         timing_begin(p, st);
     else
         p->timing.count = 0;
-    if (!p->abs_mode && p->n > 0) {
+    if (!p->abs_mode && p->n > 0 && !given_range) {
         RangeArgs ra{d_in, p->n, p->partials, p->range_counter, p->range};
         timing_mark(p, st, true, "range");
         eblc_status_t s = cuda_status(launch_range(ra, p->range_grid, st), "range launch");
@@ -299,7 +338,8 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
     ea.block = p->block;
     ea.abs_mode = p->abs_mode;
     ea.bound = p->bound;
-    ea.range = p->range;
+    ea.range = given_range ? given_range : p->range;
+    ea.range_given = given_range ? 1 : 0;
     ea.status = p->status;
     ea.ntiles = p->ntiles;
     ea.epoch = &p->d_rb->epoch;
@@ -308,6 +348,12 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
     ea.outlier_cap = p->outlier_cap;
     ea.stall_tile = (p->calls++ == p->stall_call) ? p->stall_tile : -1;
     ea.wait_ns = p->wait_ns;
+    ea.nd = p->nd;
+    for (int d = 0; d < 3; ++d) ea.dims[d] = p->dims[d];
+    if (p->nd && p->n > 0) {
+        eblc_status_t t = encode_tensor_map(p, d_in, &ea.tmap);
+        if (t != EBLC_OK) return t;
+    }
     timing_mark(p, st, true, "encode");
     eblc_status_t s = cuda_status(launch_encode(ea, p->num_sms, st), "encode launch");
     timing_mark(p, st, false, nullptr);
@@ -329,7 +375,7 @@ eblc_status_t finish_compress(eblc_plan_s *p, size_t *compressed_bytes, void *h_
         eblc_sidecar_t sc{};
         sc.magic = kMagic;
         sc.version = (uint16_t)kVersion;
-        sc.flags = (uint16_t)(p->abs_mode ? kFlagAbs : 0);
+        sc.flags = (uint16_t)((p->abs_mode ? kFlagAbs : 0) | (p->nd ? kFlagLorenzoNd : 0));
         sc.block = p->block;
         sc.chunk = kChunk;
         sc.n = p->n;
@@ -344,6 +390,7 @@ eblc_status_t finish_compress(eblc_plan_s *p, size_t *compressed_bytes, void *h_
         std::memcpy(h_sidecar, &sc, sizeof(sc));
     }
     if (err & kErrTimeout) return EBLC_TIMEOUT;
+    if (err & kErrRange) return EBLC_INVALID_ARG;
     if (err & kErrCapacity) return EBLC_CAPACITY;
     if (err & kErrCorrupt) return EBLC_CORRUPT;
     return EBLC_OK;
@@ -359,6 +406,7 @@ eblc_status_t check_stream(const eblc_plan_s *p, const eblc_sidecar_t &sc, size_
                            StreamInfo *info) {
     if (sc.magic != kMagic || sc.version != kVersion || sc.chunk != kChunk) return EBLC_CORRUPT;
     if (sc.n != p->n || sc.block != p->block) return EBLC_INVALID_ARG;
+    if (((sc.flags & kFlagLorenzoNd) != 0) != (p->nd != 0)) return EBLC_INVALID_ARG;  // the plan's predictor
     if (sc.payload_words > sc.n || sc.n_outliers > sc.n) return EBLC_CORRUPT;
     const uint64_t total = p->L.record_off + 4 * (sc.payload_words + 2 * sc.n_outliers);
     if (total != sc.total_bytes || compressed_bytes < total) return EBLC_CORRUPT;
@@ -451,6 +499,22 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
         return s;
     }
     p->n = n;
+    if (p->nd) {  // multi-dimensional Lorenzo: rank 2 or 3, dims multiples of the brick, block 64 or 256
+        const int r = rank;
+        const uint64_t be = (r == 3) ? 16 : 64;
+        bool ok = (r == 2 || r == 3) && (p->block == 64 || p->block == 256);
+        for (int i = 0; ok && i < r; ++i) ok = dims[i] > 0 && (uint64_t)dims[i] % be == 0;
+        if (!ok) {
+            EBLC_LOG("lorenzo=nd needs rank 2 or 3, block 64 or 256, dims multiples of %s",
+                     r == 3 ? "16" : "64");
+            delete p;
+            return EBLC_UNSUPPORTED;
+        }
+        p->nd = r;
+        p->dims[0] = (r == 3) ? (uint64_t)dims[0] : 1;
+        p->dims[1] = (uint64_t)dims[r - 2];
+        p->dims[2] = (uint64_t)dims[r - 1];
+    }
     p->outlier_cap = std::min<uint64_t>(p->outlier_cap, n);
     p->L = stream_layout(n, p->block);
     p->max_bytes = p->L.record_off + 4 * (n + 2 * p->outlier_cap);
@@ -594,6 +658,45 @@ EBLC_API eblc_status_t eblc_compress_async(eblc_plan_t p, const eblc_execution_t
     return s;
 }
 
+EBLC_API eblc_status_t eblc_value_range(eblc_plan_t p, const eblc_execution_t *exec, const float *d_in,
+                                        float *d_range) {
+    if (!p || !exec || !d_range) return EBLC_INVALID_ARG;
+    if (exec->kind == EBLC_EXECUTION_HIP || exec->kind == EBLC_EXECUTION_HOST) return EBLC_UNSUPPORTED;
+    if (exec->kind != EBLC_EXECUTION_CUDA) return EBLC_INVALID_ARG;
+    if ((p->n && !d_in) || (d_in && !aligned16(d_in)) || (reinterpret_cast<uintptr_t>(d_range) & 3u))
+        return EBLC_INVALID_ARG;
+    DeviceGuard g(p->device);
+    if (!g.ok) return EBLC_CUDA_ERROR;
+    cudaStream_t st = static_cast<cudaStream_t>(exec->stream);
+    if (p->n == 0) return cuda_status(cudaMemsetAsync(d_range, 0, 2 * sizeof(float), st), "range clear");
+    RangeArgs ra{d_in, p->n, p->partials, p->range_counter, d_range};
+    return cuda_status(launch_range(ra, p->range_grid, st), "range launch");
+}
+
+EBLC_API eblc_status_t eblc_compress_range(eblc_plan_t p, const eblc_execution_t *exec, const float *d_in,
+                                           const float *d_range, void *d_out, size_t out_capacity,
+                                           size_t *compressed_bytes, void *h_sidecar) {
+    if (!p || !exec || !d_range) return EBLC_INVALID_ARG;
+    if (compressed_bytes) *compressed_bytes = 0;
+    if (exec->kind == EBLC_EXECUTION_HIP || exec->kind == EBLC_EXECUTION_HOST) return EBLC_UNSUPPORTED;
+    if (exec->kind != EBLC_EXECUTION_CUDA) return EBLC_INVALID_ARG;
+    if (p->abs_mode) return EBLC_INVALID_ARG;  // a value range only matters for a relative bound
+    if (!d_out || (p->n && !d_in)) return EBLC_INVALID_ARG;
+    if (!aligned16(d_out) || (d_in && !aligned16(d_in)) || (reinterpret_cast<uintptr_t>(d_range) & 3u))
+        return EBLC_INVALID_ARG;
+    if (h_sidecar && (reinterpret_cast<uintptr_t>(h_sidecar) % kSidecarAlignment)) return EBLC_INVALID_ARG;
+    if (out_capacity < p->L.record_off) return EBLC_CAPACITY;
+    DeviceGuard g(p->device);
+    if (!g.ok) return EBLC_CUDA_ERROR;
+    cudaStream_t st = static_cast<cudaStream_t>(exec->stream);
+    eblc_status_t s;
+    if ((s = enqueue_compress(p, st, d_in, static_cast<uint8_t *>(d_out), out_capacity, true, nullptr, d_range)) !=
+        EBLC_OK)
+        return s;
+    if ((s = cuda_status(cudaStreamSynchronize(st), "compress sync")) != EBLC_OK) return s;
+    return finish_compress(p, compressed_bytes, h_sidecar);
+}
+
 EBLC_API eblc_status_t eblc_decompress(eblc_plan_t p, const eblc_execution_t *exec, const void *d_in,
                                        size_t compressed_bytes, const void *h_sidecar, float *d_out) {
     if (!p || !exec) return EBLC_INVALID_ARG;
@@ -632,6 +735,8 @@ EBLC_API eblc_status_t eblc_decompress(eblc_plan_t p, const eblc_execution_t *ex
     da.step = info.step;
     da.err = p->dec_err;
     da.wait_ns = p->wait_ns;
+    da.nd = p->nd;
+    for (int d = 0; d < 3; ++d) da.dims[d] = p->dims[d];
     if (!host) {
         da.in = static_cast<const uint8_t *>(d_in);
         da.out = d_out;

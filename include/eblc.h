@@ -110,7 +110,8 @@ typedef struct {
 typedef struct {
     uint32_t magic;         /* 0x434C4245 ("EBLC")                   */
     uint16_t version;       /* stream version (1)                    */
-    uint16_t flags;         /* bit0: absolute bound                  */
+    uint16_t flags;         /* bit0: absolute bound; bit1: 2-D / 3-D
+                               Lorenzo (lorenzo=nd)                  */
     uint32_t block;         /* B                                     */
     uint32_t chunk;         /* 4096                                  */
     uint64_t n;             /* elements                              */
@@ -144,7 +145,8 @@ EBLC_API const char *eblc_status_string(eblc_status_t status);
  * Create a plan for float32 snapshots of shape dims[0..rank) (slowest to
  * fastest).  strides (in elements, slowest to fastest) may be NULL for
  * C-contiguous data; any non-contiguous stride gives EBLC_UNSUPPORTED.  The
- * data are coded as one flat sequence in C order.  Requires 1 <= rank <= 8,
+ * data are coded as one flat sequence in C order (unless lorenzo=nd, below).
+ * Requires 1 <= rank <= 8,
  * dims >= 0 and n = prod(dims) <= 2^30.
  *
  * options: NULL -> relative bound 1e-4, block 128.  A bare decimal ("1e-3")
@@ -155,6 +157,13 @@ EBLC_API const char *eblc_status_string(eblc_status_t status);
  *   block=<B>        32 | 64 | 128 | 256 (default 128)
  *   outlier_cap=<k>  most outliers per stream (default n); more gives
  *                    EBLC_CAPACITY
+ *   lorenzo=nd       2-D / 3-D Lorenzo predictor over the plan's own dims
+ *                    (rank 2 {Y, X} or rank 3 {Z, Y, X}, each a multiple of 64
+ *                    (2-D) or 16 (3-D); block 64 or 256, i.e. 8x8 / 16x16
+ *                    or 4x4x4 / 4x8x8 elements), reset at every block face;
+ *                    bricks of 64x64 or 16x16x16 elements take the place of
+ *                    the 4096-element chunks.  Otherwise EBLC_UNSUPPORTED.
+ *                    Default lorenzo=1d: the data coded as one flat sequence
  *   timing=1         record per-kernel device times (eblc_plan_kernel_times)
  *   wait_ms=<t>      limit of device-side waits in milliseconds (default 2000)
  *   stall_tile=<t>   test hook: tile t of one compress call never publishes
@@ -228,6 +237,48 @@ typedef struct eblc_async_result_t {
  */
 EBLC_API eblc_status_t eblc_compress_async(eblc_plan_t plan, const eblc_execution_t *exec, const float *d_in,
                                            void *d_out, size_t out_capacity, eblc_async_result_t *d_result);
+
+/*
+ * Value range of one snapshot: d_range[0] = vmin, d_range[1] = vmax over the
+ * finite elements of d_in (each +0 where the value is a zero; both 0 when no
+ * element is finite, or n = 0).  This is the range a relative bound is
+ * relative to ("Pipeline specialization internals", Priming: the value-range
+ * scan that resolves the bound before the fused kernel).
+ *   d_in     n float32 values in device memory, 16-byte aligned
+ *   d_range  device float[2], 4-byte aligned, caller owned
+ * CUDA kind only (HOST and HIP: EBLC_UNSUPPORTED).  Queued on exec->stream;
+ * no synchronisation.  Uses the plan's scratch, like its other calls.
+ *
+ * With eblc_compress_range this codes an array split across processes (one
+ * contiguous part per GPU) under one relative bound: each process computes
+ * its part's range here, the processes combine them (minimum of vmin,
+ * maximum of vmax: one small all-reduce, which is the caller's, e.g. NCCL
+ * through torch.distributed), and each compresses its part under the
+ * combined range ("DevitoComp provider interface", Validating a private
+ * provider: the provider runs inside an MPI-run consumer).
+ */
+EBLC_API eblc_status_t eblc_value_range(eblc_plan_t plan, const eblc_execution_t *exec, const float *d_in,
+                                        float *d_range);
+
+/*
+ * eblc_compress with the value range given instead of taken from d_in: the
+ * bound is eb = rel * (vmax - vmin) with {vmin, vmax} = d_range[0..1] read
+ * from device memory by the encoder (relative-bound plans only, else
+ * EBLC_INVALID_ARG).  Meant for one part of a larger array, with the range of
+ * the whole (see eblc_value_range); outlier indices in the stream count from
+ * the part's first element, and the stream decodes on its own with
+ * eblc_decompress.  When the parts are cut at multiples of 4096 elements,
+ * their width bytes, payload words and outlier values are those of the whole
+ * array's stream for the same chunks.
+ *   d_range  device float[2], 4-byte aligned; must be finite with
+ *            vmin <= vmax, else the call returns EBLC_INVALID_ARG (checked
+ *            on the device, reported after the closing synchronisation)
+ * Other arguments, synchronisation and sidecar as for eblc_compress; CUDA
+ * kind only.
+ */
+EBLC_API eblc_status_t eblc_compress_range(eblc_plan_t plan, const eblc_execution_t *exec, const float *d_in,
+                                           const float *d_range, void *d_out, size_t out_capacity,
+                                           size_t *compressed_bytes, void *h_sidecar);
 
 /*
  * Decompress one snapshot.
