@@ -410,6 +410,93 @@ def run_ours(args):
     return 0
 
 
+def run_sharded(args):
+    """One array split across the ranks (chunk-aligned contiguous parts, one
+    per GPU), each step: every rank's value range, one NCCL all-reduce of the
+    ranges, each rank's compress under the combined range, the stream-size
+    exchange, then each rank's decompress.  Strong scaling: the whole job
+    processes the workload once per step.  CUDA events around the calls,
+    median step, max over ranks."""
+    import torch
+
+    import error_bounded_lossy_encode_b200 as E
+    from error_bounded_lossy_encode_b200 import sharded as SH
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x_np, block, mode, bound = workload(args.workload, args.elements, args.rel, args.abs, args.block)
+    if mode != "rel":
+        raise SystemExit("--sharded needs a relative bound (the range all-reduce is its only exchange)")
+    a, b = SH.part_bounds(x_np.size, world, rank)
+    part = np.ascontiguousarray(x_np[a:b])
+    st, plan = E.eblc_plan_create([part.size], None, options_string(block, mode, bound))
+    if st != E.EBLC_OK:
+        raise RuntimeError("plan_create: " + E.STATUS_NAMES[st])
+    _, lim = E.eblc_plan_get_limits(plan)
+    cap = lim["max_compressed_bytes"]
+    x = torch.from_numpy(part).to(dev)
+    out = torch.empty(cap, dtype=torch.uint8, device=dev)
+    y = torch.empty(max(part.size, 1), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ex = E.cuda_exec(stream.cuda_stream)
+
+    def step():
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.fill_(1)
+        ev[0].record(stream)
+        st, nb, off, total, rng = SH.compress_part(plan, x, out, cap)
+        ev[1].record(stream)
+        if st != E.EBLC_OK:
+            raise RuntimeError("compress_part: " + E.STATUS_NAMES[st])
+        flush.fill_(2)
+        ev[2].record(stream)
+        if E.eblc_decompress(plan, ex, out.data_ptr(), nb, None, y.data_ptr()) != E.EBLC_OK:
+            raise RuntimeError("decompress")
+        ev[3].record(stream)
+        return ev, nb, total
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+    recs = [step() for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    steps = [r[0][0].elapsed_time(r[0][1]) / 1e3 + r[0][2].elapsed_time(r[0][3]) / 1e3 for r in recs]
+    (t_step,) = max_over_ranks([float(np.median(steps))], world, dev)
+    total = recs[-1][2]
+    if rank == 0:
+        line = {"metric": METRIC, "value": round(4.0 * x_np.size / t_step / 1e9, 2), "unit": "GB/s",
+                "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup),
+                "ms_per_step": round(1e3 * t_step, 4), "higher_is_better": True, "scaling": "strong",
+                "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                "config": dict(workload_config(args, x_np.size, block, mode, bound, world),
+                               parallelism=f"sharded{world}"),
+                "timing": "CUDA events around value range + range all-reduce + compress under the combined range + "
+                          "size exchange, and around decompress; median step, max over ranks",
+                "ratio": round(4.0 * x_np.size / total, 4), "stream_bytes_all_ranks": int(total),
+                "gpu_launches": 4 * args.steps}
+        print(json.dumps(line), flush=True)
+    E.eblc_plan_destroy(plan)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def run_graph_compress(E, plan, x, out, cap, flush, nbytes, args, world, dev):
     """Compress captured once into a CUDA graph (eblc_compress_async: no host
     synchronisation inside) and replayed; CUDA events around each replay, L2
@@ -560,9 +647,13 @@ def main(argv=None):
     ap.add_argument("--rel", type=float, default=None, help="override the workload's bound: relative")
     ap.add_argument("--abs", type=float, default=None, help="override the workload's bound: absolute")
     ap.add_argument("--block", type=int, default=None, choices=(32, 64, 128, 256), help="override the block size")
+    ap.add_argument("--sharded", action="store_true",
+                    help="split one array across the ranks (range all-reduce; strong scaling) instead of replicas")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.sharded:
+        return run_sharded(args)
     return run_ours(args)
 
 
