@@ -108,6 +108,18 @@ def lib():
         L.orc_lorenzo_block.restype = None
         L.orc_unlorenzo_block.argtypes = [P, P, P]
         L.orc_unlorenzo_block.restype = None
+        L.orc_bitshuffle.argtypes = [P, u32, P]
+        L.orc_bitshuffle.restype = None
+        L.orc_unbitshuffle.argtypes = [P, u32, P]
+        L.orc_unbitshuffle.restype = None
+        L.orc_rze.argtypes = [P, u32, P]
+        L.orc_rze.restype = u32
+        L.orc_unrze.argtypes = [P, u64, u32, P]
+        L.orc_unrze.restype = ctypes.c_int64
+        L.orc_max_chunked_bytes.argtypes = [u64, u32, u64]
+        L.orc_max_chunked_bytes.restype = u64
+        L.orc_compress_chunked.argtypes = [P, u64, u32, ctypes.c_int, dbl, u64, P, u64]
+        L.orc_compress_chunked.restype = ctypes.c_int64
         L.orc_decompress.argtypes = [P, u64, P, u64]
         L.orc_decompress.restype = ctypes.c_int
         L.orc_block_codes.argtypes = [P, u64, u32, flt, P, P]
@@ -351,3 +363,59 @@ def decompress_omp(stream, n: int) -> np.ndarray:
     if rc != 0:
         raise OracleError(rc)
     return out[:n]
+
+
+def bitshuffle(words) -> np.ndarray:
+    """Bit-plane transpose of a multiple of 32 codes (see orc_bitshuffle)."""
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    out = np.zeros(max(w.size, 1), np.uint32)
+    lib().orc_bitshuffle(_ptr(w), w.size, _ptr(out))
+    return out[: w.size]
+
+
+def unbitshuffle(words) -> np.ndarray:
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    out = np.zeros(max(w.size, 1), np.uint32)
+    lib().orc_unbitshuffle(_ptr(w), w.size, _ptr(out))
+    return out[: w.size]
+
+
+def rze(words) -> np.ndarray:
+    """Zero elimination: bitmap words, then the nonzero words."""
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    out = np.zeros(max(w.size + w.size // 32, 1), np.uint32)
+    k = lib().orc_rze(_ptr(w), w.size, _ptr(out))
+    return out[:k]
+
+
+def unrze(words, mp: int):
+    """Inverse of rze for mp words; returns (words, consumed) or raises."""
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    src = w if w.size else np.zeros(1, np.uint32)
+    out = np.zeros(max(mp, 1), np.uint32)
+    k = lib().orc_unrze(_ptr(src), w.size, mp, _ptr(out))
+    if k < 0:
+        raise OracleError(int(k))
+    return out[:mp], int(k)
+
+
+def max_chunked_bytes(n: int, chunk_bytes: int, outlier_cap: int | None = None) -> int:
+    return int(lib().orc_max_chunked_bytes(n, chunk_bytes, n if outlier_cap is None else outlier_cap))
+
+
+def compress_chunked(x, chunk_bytes: int = 16384, *, rel: float | None = None, abs: float | None = None,
+                     outlier_cap: int | None = None):
+    """The chunk-cooperative codec (Quant -> Diff -> Bitshuffle -> RZE, see
+    orc_compress_chunked): the stream as a uint8 array."""
+    x = _f32(x).reshape(-1)
+    if (rel is None) == (abs is None):
+        raise ValueError("exactly one of rel / abs")
+    abs_mode = abs is not None
+    cap = x.size if outlier_cap is None else int(outlier_cap)
+    need = max(max_chunked_bytes(x.size, chunk_bytes, cap), 1)
+    out = np.zeros(need, np.uint8)
+    rc = lib().orc_compress_chunked(_ptr(x), x.size, chunk_bytes, int(abs_mode), float(abs if abs_mode else rel),
+                                    cap, _ptr(out), need)
+    if rc < 0:
+        raise OracleError(int(rc))
+    return out[:rc].copy()

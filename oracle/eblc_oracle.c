@@ -81,6 +81,7 @@
 #define ORC_HEADER_BYTES 128u
 #define ORC_FLAG_ABS 1u
 #define ORC_FLAG_LORENZO_ND 2u    /* 2-D / 3-D Lorenzo over the array's own dims */
+#define ORC_FLAG_CHUNKED 4u       /* chunk-cooperative codec: Diff -> Bitshuffle -> RZE */
 
 /* error codes returned as negative values */
 #define ORC_ERR_ARG (-1)
@@ -662,6 +663,19 @@ int orc_parse_header(const uint8_t *s, uint64_t bytes, orc_header *h) {
     h->dims[0] = get_u64(s + 96);
     h->dims[1] = get_u64(s + 104);
     h->dims[2] = get_u64(s + 112);
+    if (h->flags & ORC_FLAG_CHUNKED) {
+        if (h->magic != ORC_MAGIC || h->version != ORC_VERSION || h->block != 0 ||
+            (h->chunk != 1024 && h->chunk != 2048 && h->chunk != 4096) || (h->flags & ORC_FLAG_LORENZO_ND) ||
+            h->n > ORC_MAX_N || h->nb != 0 || h->nc != (h->n + h->chunk - 1) / h->chunk ||
+            h->W > h->n + 32 * h->nc || h->m > h->n || h->dims[0] || h->dims[1] || h->dims[2])
+            return ORC_ERR_CORRUPT;
+        orc_layout L = layout_of(0, h->nc, h->W, h->m);
+        if (L.total != h->total || h->total > bytes) return ORC_ERR_CORRUPT;
+        h->width_off = L.width_off;
+        h->index_off = L.index_off;
+        h->record_off = L.record_off;
+        return 0;
+    }
     if (h->magic != ORC_MAGIC || h->version != ORC_VERSION || !block_ok(h->block) ||
         h->chunk != ORC_CHUNK)
         return ORC_ERR_CORRUPT;
@@ -689,6 +703,7 @@ int orc_parse_header(const uint8_t *s, uint64_t bytes, orc_header *h) {
  * undelta -> dequant code * 2eb), then each chunk's outliers are written
  * back over the reconstruction.                                            */
 static int decompress_nd(const uint8_t *s, const orc_header *h, float *out);
+static int decompress_chunked(const uint8_t *s, const orc_header *h, float *out);
 
 int orc_decompress(const uint8_t *s, uint64_t bytes, float *out, uint64_t n_expected) {
     orc_header h;
@@ -696,6 +711,7 @@ int orc_decompress(const uint8_t *s, uint64_t bytes, float *out, uint64_t n_expe
     if (rc != 0) return rc;
     if (h.n != n_expected) return ORC_ERR_ARG;
     if (h.flags & ORC_FLAG_LORENZO_ND) return decompress_nd(s, &h, out);
+    if (h.flags & ORC_FLAG_CHUNKED) return decompress_chunked(s, &h, out);
 
     uint32_t words[256], z[256];
     uint64_t blocks_per_chunk = ORC_CHUNK / h.block;
@@ -783,6 +799,232 @@ static int decompress_nd(const uint8_t *s, const orc_header *h, float *out) {
             if (i >= h->n || zz < z0 || zz >= z0 + ce[0] || yy < y0 || yy >= y0 + ce[1] || xx < x0 ||
                 xx >= x0 + ce[2])
                 return ORC_ERR_CORRUPT;
+            memcpy(&out[i], &bits, 4);
+        }
+    }
+    if (W_seen != h->W) return ORC_ERR_CORRUPT;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Chunk-cooperative codec ("Pipeline specialization internals",
+ * Chunk-cooperative path: one CTA owns a byte chunk of 4096, 8192 or 16384
+ * bytes, a Quant -> Diff -> Bitshuffle -> RZE chain; "nvrtc_chunk_fusion.h
+ * File Reference", launchNvrtcChunkFusedEncode: each chunk's coded form lands
+ * in a scratch slot of CHUNK_BYTES with its size, then a cross-chunk scan
+ * packs them into one archive, the outliers leaving through a side list).
+ * The pages name the ops and give no definitions; readings:
+ *   - chunk: CHUNK_BYTES of float32 input, m = CHUNK_BYTES / 4 elements (the
+ *     last chunk may be shorter);
+ *   - Quant: the linear quantizer and outlier rule of the main path;
+ *   - Diff: first difference of the codes within the chunk (0 before its
+ *     first code), taken to zigzag form so that small differences of either
+ *     sign leave the high bit planes zero;
+ *   - Bitshuffle: the chunk's codes, zero-padded to mp = a multiple of 32, in
+ *     groups of 32; bit b of code l of group g is bit l of word b*(mp/32) + g
+ *     (32 bit planes, each mp/32 words);
+ *   - RZE (zero elimination): one bitmap bit per shuffled word (bit j of the
+ *     bitmap: word j is not zero; mp/32 bitmap words, least significant bit
+ *     first), then the nonzero words in order;
+ *   - a chunk whose RZE form is not smaller than its mp shuffled words keeps
+ *     the shuffled words verbatim, so a coded chunk never exceeds its input;
+ *   - record of a chunk: one word P | raw << 31 (P payload words follow),
+ *     the payload, then the chunk's outlier indices and values (ascending
+ *     index), located by the chunk index as in the main format.          */
+void orc_bitshuffle(const uint32_t *in, uint32_t mp, uint32_t *out) {
+    uint32_t G = mp / 32;
+    for (uint32_t b = 0; b < 32; ++b)
+        for (uint32_t g = 0; g < G; ++g) {
+            uint32_t word = 0;
+            for (uint32_t l = 0; l < 32; ++l) word |= ((in[g * 32 + l] >> b) & 1u) << l;
+            out[b * G + g] = word;
+        }
+}
+
+void orc_unbitshuffle(const uint32_t *in, uint32_t mp, uint32_t *out) {
+    uint32_t G = mp / 32;
+    for (uint32_t g = 0; g < G; ++g)
+        for (uint32_t l = 0; l < 32; ++l) {
+            uint32_t code = 0;
+            for (uint32_t b = 0; b < 32; ++b) code |= ((in[b * G + g] >> l) & 1u) << b;
+            out[g * 32 + l] = code;
+        }
+}
+
+/* Zero elimination of mp words (mp a multiple of 32): returns the words
+ * written to out (mp / 32 bitmap words, then the nonzero words).           */
+uint32_t orc_rze(const uint32_t *in, uint32_t mp, uint32_t *out) {
+    uint32_t nbm = mp / 32, k = nbm;
+    for (uint32_t i = 0; i < nbm; ++i) out[i] = 0;
+    for (uint32_t j = 0; j < mp; ++j)
+        if (in[j] != 0) {
+            out[j / 32] |= 1u << (j % 32);
+            out[k++] = in[j];
+        }
+    return k;
+}
+
+/* Inverse: from `avail` words at in, mp words to out.  Returns the words
+ * consumed, or -1 if the bitmap calls for more words than avail.           */
+int64_t orc_unrze(const uint32_t *in, uint64_t avail, uint32_t mp, uint32_t *out) {
+    uint32_t nbm = mp / 32;
+    if (avail < nbm) return -1;
+    uint64_t k = nbm;
+    for (uint32_t j = 0; j < mp; ++j) {
+        if ((in[j / 32] >> (j % 32)) & 1u) {
+            if (k >= avail) return -1;
+            out[j] = in[k++];
+        } else {
+            out[j] = 0;
+        }
+    }
+    return (int64_t)k;
+}
+
+static int chunk_bytes_ok(uint32_t cb) { return cb == 4096 || cb == 8192 || cb == 16384; }
+
+uint64_t orc_max_chunked_bytes(uint64_t n, uint32_t chunk_bytes, uint64_t outlier_cap) {
+    if (!chunk_bytes_ok(chunk_bytes)) return 0;
+    uint64_t m = chunk_bytes / 4, nc = (n + m - 1) / m;
+    return layout_of(0, nc, nc + n + 31 * nc, outlier_cap).total;
+}
+
+int64_t orc_compress_chunked(const float *x, uint64_t n, uint32_t chunk_bytes, int abs_mode, double bound,
+                             uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
+    if (!chunk_bytes_ok(chunk_bytes) || !(bound >= 0.0) || !isfinite(bound)) return ORC_ERR_ARG;
+    if (n > ORC_MAX_N) return ORC_ERR_ARG;
+    if (fegetround() != FE_TONEAREST) return ORC_ERR_ARG;
+    float vmin = 0.0f, vmax = 0.0f;
+    if (!abs_mode) orc_value_range(x, n, &vmin, &vmax);
+    double eb;
+    float inv2eb, step;
+    orc_resolve_bound(abs_mode, bound, vmin, vmax, &eb, &inv2eb, &step);
+
+    uint32_t mc_max = chunk_bytes / 4;
+    uint64_t nc = (n + mc_max - 1) / mc_max;
+    int32_t *q = (int32_t *)malloc((n ? n : 1) * sizeof(int32_t));
+    uint8_t *flag = (uint8_t *)malloc(n ? n : 1);
+    uint32_t *d = (uint32_t *)malloc(4096 * 4), *sh = (uint32_t *)malloc(4096 * 4);
+    uint32_t *rz = (uint32_t *)malloc((4096 + 128) * 4);
+    if (!q || !flag || !d || !sh || !rz) {
+        free(q); free(flag); free(d); free(sh); free(rz);
+        return ORC_ERR_NOMEM;
+    }
+    orc_quantize(x, n, inv2eb, step, eb, q, flag);
+    uint64_t m = 0, W = 0;
+    for (uint64_t i = 0; i < n; ++i) m += flag[i];
+    for (int pass = 0; pass < 2; ++pass) {
+        /* pass 0 sizes every chunk; pass 1 writes the stream */
+        orc_layout L = layout_of(0, nc, W, m);
+        if (pass == 1) {
+            int64_t status = (int64_t)L.total;
+            if (m > outlier_cap) status = ORC_ERR_OUTLIER_CAP;
+            else if (L.total > out_cap) status = ORC_ERR_CAPACITY;
+            if (status < 0) {
+                free(q); free(flag); free(d); free(sh); free(rz);
+                return status;
+            }
+            memset(out, 0, L.total);
+            put_u32(out + 0, ORC_MAGIC);
+            put_u16(out + 4, (uint16_t)ORC_VERSION);
+            put_u16(out + 6, (uint16_t)((abs_mode ? ORC_FLAG_ABS : 0u) | ORC_FLAG_CHUNKED));
+            put_u64(out + 8, n);
+            put_u32(out + 16, 0);
+            put_u32(out + 20, mc_max);
+            put_f64(out + 24, eb);
+            put_f32(out + 32, inv2eb);
+            put_f32(out + 36, step);
+            put_f32(out + 40, vmin);
+            put_f32(out + 44, vmax);
+            put_u64(out + 48, 0);
+            put_u64(out + 56, nc);
+            put_u64(out + 64, W);
+            put_u64(out + 72, m);
+            put_u64(out + 80, L.total);
+            put_f64(out + 88, bound);
+        }
+        uint64_t rec = 0, before = 0;
+        for (uint64_t c = 0; c < nc; ++c) {
+            uint64_t e0 = c * mc_max, e1 = e0 + mc_max < n ? e0 + mc_max : n;
+            uint32_t cnt = (uint32_t)(e1 - e0), mp = (cnt + 31) / 32 * 32;
+            int32_t prev = 0;  /* Diff: 0 before the chunk's first code */
+            for (uint32_t j = 0; j < mp; ++j) {
+                if (j < cnt) {
+                    d[j] = orc_zigzag(q[e0 + j] - prev);
+                    prev = q[e0 + j];
+                } else {
+                    d[j] = 0;
+                }
+            }
+            orc_bitshuffle(d, mp, sh);
+            uint32_t r = orc_rze(sh, mp, rz);
+            int raw = r >= mp;
+            uint32_t P = raw ? mp : r;
+            uint64_t mc = 0;
+            for (uint64_t i = e0; i < e1; ++i) mc += flag[i];
+            if (pass == 0) {
+                W += 1 + P;
+                continue;
+            }
+            put_u32(out + L.index_off + 8 * c, (uint32_t)rec);
+            put_u32(out + L.index_off + 8 * c + 4, (uint32_t)before);
+            uint8_t *rp = out + L.record_off + 4 * rec;
+            put_u32(rp, P | (raw ? 0x80000000u : 0u));
+            for (uint32_t k = 0; k < P; ++k) put_u32(rp + 4 * (1 + k), raw ? sh[k] : rz[k]);
+            uint64_t k = 0;
+            for (uint64_t i = e0; i < e1; ++i) {
+                if (!flag[i]) continue;
+                uint32_t bits;
+                memcpy(&bits, &x[i], 4);
+                put_u32(rp + 4 * (1 + P + k), (uint32_t)i);
+                put_u32(rp + 4 * (1 + P + mc + k), bits);
+                ++k;
+            }
+            rec = rec + 1 + P + 2 * mc;
+            before = before + mc;
+        }
+        if (pass == 1) {
+            free(q); free(flag); free(d); free(sh); free(rz);
+            return (int64_t)L.total;
+        }
+    }
+    return ORC_ERR_ARG; /* not reached */
+}
+
+static int decompress_chunked(const uint8_t *s, const orc_header *h, float *out) {
+    uint32_t rec_words[4096 + 129], sh[4096], d[4096];
+    uint64_t R = h->W + 2 * h->m, W_seen = 0;
+    for (uint64_t c = 0; c < h->nc; ++c) {
+        uint64_t rec = get_u32(s + h->index_off + 8 * c);
+        uint64_t before = get_u32(s + h->index_off + 8 * c + 4);
+        uint64_t rec_next = (c + 1 < h->nc) ? get_u32(s + h->index_off + 8 * (c + 1)) : R;
+        uint64_t after = (c + 1 < h->nc) ? get_u32(s + h->index_off + 8 * (c + 1) + 4) : h->m;
+        if (rec_next < rec || after < before || rec_next > R || after > h->m) return ORC_ERR_CORRUPT;
+        uint64_t mc = after - before, e0 = c * h->chunk, e1 = e0 + h->chunk < h->n ? e0 + h->chunk : h->n;
+        uint32_t cnt = (uint32_t)(e1 - e0), mp = (cnt + 31) / 32 * 32;
+        if (rec_next - rec < 1 + 2 * mc) return ORC_ERR_CORRUPT;
+        uint32_t head = get_u32(s + h->record_off + 4 * rec), P = head & 0x7fffffffu;
+        int raw = (head >> 31) != 0;
+        if (1 + (uint64_t)P + 2 * mc != rec_next - rec || P > mp + mp / 32) return ORC_ERR_CORRUPT;
+        for (uint32_t k = 0; k < P; ++k) rec_words[k] = get_u32(s + h->record_off + 4 * (rec + 1 + k));
+        if (raw) {
+            if (P != mp) return ORC_ERR_CORRUPT;
+            memcpy(sh, rec_words, 4 * mp);
+        } else if (orc_unrze(rec_words, P, mp, sh) != (int64_t)P) {
+            return ORC_ERR_CORRUPT;
+        }
+        orc_unbitshuffle(sh, mp, d);
+        int64_t qv = 0; /* inverse Diff: running sum from 0 at the chunk start */
+        for (uint32_t j = 0; j < cnt; ++j) {
+            qv += orc_unzigzag(d[j]);
+            out[e0 + j] = dequant((int32_t)(uint32_t)(uint64_t)qv, h->step);
+        }
+        W_seen += 1 + P;
+        uint64_t o = rec + 1 + P;
+        for (uint64_t k = 0; k < mc; ++k) {
+            uint32_t i = get_u32(s + h->record_off + 4 * (o + k));
+            uint32_t bits = get_u32(s + h->record_off + 4 * (o + mc + k));
+            if (i < e0 || i >= e1) return ORC_ERR_CORRUPT;
             memcpy(&out[i], &bits, 4);
         }
     }

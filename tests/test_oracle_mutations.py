@@ -35,6 +35,11 @@ MUTATIONS = [
     ("Lorenzo inverse along y", "q[e] = (int32_t)((uint32_t)q[e] + (uint32_t)q[e - be[2]]);",
      "q[e] = (int32_t)((uint32_t)q[e] + (uint32_t)q[e - 1]);"),
     ("block z index", "uint64_t z = cz * ce[0] + iz * be[0] + ez;", "uint64_t z = cz * ce[0] + iz * be[0];"),
+    ("bitshuffle plane order", "out[b * G + g] = word;", "out[g * 32 + b] = word;"),
+    ("zero-elimination bitmap order", "out[j / 32] |= 1u << (j % 32);", "out[j / 32] |= 1u << (31 - j % 32);"),
+    ("chunk Diff without reset", "int32_t prev = 0;  /* Diff: 0 before the chunk's first code */",
+     "static int32_t prev = 0;  /* Diff: 0 before the chunk's first code */"),
+    ("verbatim when larger", "int raw = r >= mp;", "int raw = r > mp + 1000000;"),
 ]
 
 
@@ -42,6 +47,7 @@ def _run_pins(src_path: str) -> subprocess.CompletedProcess:
     env = dict(os.environ, EBLC_ORACLE_SRC=src_path, PYTHONDONTWRITEBYTECODE="1")
     return subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_oracle_pins.py"),
                            os.path.join(ROOT, "tests", "test_oracle_nd_pins.py"),
+                           os.path.join(ROOT, "tests", "test_oracle_chunked_pins.py"),
                            "-x", "-q", "-p", "no:cacheprovider", "-k", "not fuzz"],
                           cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
 
