@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libeblc.so")
-SOURCES = ("range.cu", "encode.cu", "decode.cu", "plan.cu", "noalloc.cu")
+SOURCES = ("range.cu", "encode.cu", "decode.cu", "chunked.cu", "plan.cu", "noalloc.cu")
 HEADERS = ("common.cuh", "kernels.h")
 
 NVCC_FLAGS = [

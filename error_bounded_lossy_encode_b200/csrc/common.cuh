@@ -19,6 +19,7 @@ constexpr uint32_t kMagic = 0x434C4245u;  // "EBLC"
 constexpr uint32_t kVersion = 1;
 constexpr uint16_t kFlagAbs = 1;
 constexpr uint16_t kFlagLorenzoNd = 2;  // 2-D / 3-D Lorenzo over the array's dims (bytes 96..119: Z, Y, X)
+constexpr uint16_t kFlagChunked = 4;    // chunk-cooperative codec (Diff -> Bitshuffle -> RZE), no block widths
 constexpr uint64_t kMaxN = 1ull << 30;
 
 // Device error word bits.
@@ -36,6 +37,18 @@ __host__ __device__ inline Layout stream_layout(uint64_t n, uint32_t block) {
     L.nc = (n + kChunk - 1) / kChunk;
     L.width_off = kHeaderBytes;
     L.index_off = L.width_off + pad16(L.nb);
+    L.record_off = L.index_off + pad16(8u * L.nc);
+    return L;
+}
+
+// Layout of a stream of the chunk-cooperative codec: no width bytes, one
+// index entry per chunk of m elements, then the chunk records.
+__host__ __device__ inline Layout chunked_layout(uint64_t n, uint32_t m) {
+    Layout L;
+    L.nb = 0;
+    L.nc = (n + m - 1) / m;
+    L.width_off = kHeaderBytes;
+    L.index_off = kHeaderBytes;
     L.record_off = L.index_off + pad16(8u * L.nc);
     return L;
 }
@@ -160,29 +173,10 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
         : "memory");
 }
 
-// Bulk prefetch of [src, src + bytes) into L2 (no completion, no shared
-// memory): puts more DRAM reads in flight than the shared-memory stages can
-// hold.  src 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// 16-byte asynchronous copy global -> shared through L1 (cp.async), and the
-// arrive-on of an mbarrier once all of this thread's earlier cp.async have
-// landed (the mbarrier's expected count includes these arrivals).
-__device__ __forceinline__ void async_copy16(void *dst_smem, const void *src_gmem) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src_gmem) : "memory");
-}
-
-__device__ __forceinline__ void async_copy_arrive(uint64_t *bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // Tiled tensor copies global -> shared (one box of the tensor map at the
-// given element coordinates, x innermost) completing on an mbarrier, and
-// their L2 prefetch form.  The x coordinate times 4 bytes is a multiple of
-// 16 at every call site (bricks start at multiples of 16 elements).  Never
-// used with .multicast.
+// given element coordinates, x innermost) completing on an mbarrier.  The x
+// coordinate times 4 bytes is a multiple of 16 at every call site (bricks
+// start at multiples of 16 elements).  Never used with .multicast.
 __device__ __forceinline__ void tensor_g2s_3d(void *dst_smem, const void *tmap, int x, int y, int z, uint64_t *bar) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
@@ -197,20 +191,6 @@ __device__ __forceinline__ void tensor_g2s_2d(void *dst_smem, const void *tmap, 
         "[%4];" ::"r"(smem_u32(dst_smem)),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
-}
-
-__device__ __forceinline__ void tensor_prefetch_3d(const void *tmap, int x, int y, int z) {
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(tmap)),
-                 "r"(x), "r"(y), "r"(z)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tensor_prefetch_2d(const void *tmap, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                     reinterpret_cast<uint64_t>(tmap)),
-                 "r"(x), "r"(y)
-                 : "memory");
 }
 
 // Brick t of a multi-dimensional array {Z, Y, X} in C order over the brick

@@ -84,4 +84,40 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs &a, int num_sms, cudaStream_t stream);
 
+// Chunk-cooperative codec (Quant -> Diff -> Bitshuffle -> RZE): chunks of m
+// = 1024, 2048 or 4096 elements.  One launch sequence writes the stream:
+// encode (each chunk's record into its scratch slot of chunked_slot_words(m)
+// words, its size and outlier count), scan (chunk index, header, result
+// block), gather (records to their offsets).
+struct ChunkedArgs {
+    const float *in;          // n floats
+    uint64_t n;
+    uint32_t m;               // elements per chunk
+    uint64_t nc;
+    int abs_mode;
+    double bound;
+    const float *range;       // vmin, vmax (relative mode)
+    uint32_t *scratch;        // nc slots
+    uint32_t slot_words;
+    uint32_t *sizes, *outl, *offs;  // nc each: record words, outliers, record word offset
+    uint8_t *out;
+    uint64_t out_cap;
+    uint64_t *result;         // as EncodeArgs::result
+    uint32_t *err;
+    uint64_t outlier_cap;
+};
+uint64_t chunked_slot_words(uint32_t m);
+cudaError_t launch_chunked_encode(const ChunkedArgs &a, int num_sms, cudaStream_t stream);
+
+struct ChunkedDecArgs {
+    const uint8_t *in;        // stream, 16-byte aligned
+    uint64_t n;
+    uint32_t m;
+    uint64_t W, mo;           // payload words (record head words included) and outliers
+    float step;
+    float *out;
+    uint32_t *err;
+};
+cudaError_t launch_chunked_decode(const ChunkedDecArgs &a, int num_sms, cudaStream_t stream);
+
 }  // namespace eblc

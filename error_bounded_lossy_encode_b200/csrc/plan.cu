@@ -85,6 +85,10 @@ struct eblc_plan_s {
     uint64_t wait_ns = 2000ull * 1000000ull;
     int64_t stall_tile = -1;
     int nd = 0;                     // option lorenzo=nd: 2 or 3 (the plan's rank), 0 for the 1-D path
+    uint32_t chunked_m = 0;         // option codec=chunked: elements per chunk (1024, 2048, 4096), else 0
+    int opt_chunked = 0;            // options as parsed (resolved by plan_create)
+    uint32_t opt_chunk_bytes = 0;
+    uint32_t *chunk_scratch = nullptr;  // codec=chunked: nc record slots, then sizes, outlier counts, offsets
     uint64_t dims[3] = {0, 0, 0};   // {Z, Y, X} of a multi-dimensional plan (Z = 1 for 2-D)
     uint64_t stall_call = 0;        // the compress call (0-based) that stall_tile applies to
     uint64_t calls = 0;             // compress calls enqueued so far
@@ -198,6 +202,13 @@ eblc_status_t parse_options(const char *options, eblc_plan_s *p, bool *timing) {
         } else if (key == "outlier_cap") {
             if (!parse_int(val, &iv) || iv < 0) return EBLC_INVALID_ARG;
             p->outlier_cap = (uint64_t)iv;  // clamped to n by the caller
+        } else if (key == "codec") {
+            if (val == "chunked") p->opt_chunked = 1;
+            else if (val != "lorenzo") return EBLC_INVALID_ARG;
+        } else if (key == "chunk") {  // bytes of float32 input per chunk of the chunked codec
+            if (!parse_int(val, &iv)) return EBLC_INVALID_ARG;
+            if (iv != 4096 && iv != 8192 && iv != 16384) return EBLC_UNSUPPORTED;
+            p->opt_chunk_bytes = (uint32_t)iv;
         } else if (key == "lorenzo") {
             if (val == "nd") p->nd = -1;  // resolved against the dims by the caller
             else if (val != "1d") return EBLC_INVALID_ARG;
@@ -234,6 +245,7 @@ void destroy(eblc_plan_s *p) {
     for (cudaEvent_t &e : p->timing.ev)
         if (e) cudaEventDestroy(e);
     if (p->scratch) cudaFree(p->scratch);
+    if (p->chunk_scratch) cudaFree(p->chunk_scratch);
     if (p->stage_in) cudaFree(p->stage_in);
     if (p->stage_out) cudaFree(p->stage_out);
     if (p->host_stream) cudaStreamDestroy(p->host_stream);
@@ -330,6 +342,38 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
         timing_mark(p, st, false, nullptr);
         if (s != EBLC_OK) return s;
     }
+    if (p->chunked_m) {
+        const uint64_t slot = chunked_slot_words(p->chunked_m);
+        ChunkedArgs ca{};
+        ca.in = d_in;
+        ca.n = p->n;
+        ca.m = p->chunked_m;
+        ca.nc = p->L.nc;
+        ca.abs_mode = p->abs_mode;
+        ca.bound = p->bound;
+        ca.range = given_range ? given_range : p->range;
+        ca.scratch = p->chunk_scratch;
+        ca.slot_words = (uint32_t)slot;
+        ca.sizes = p->chunk_scratch ? p->chunk_scratch + p->L.nc * slot : nullptr;
+        ca.outl = ca.sizes ? ca.sizes + p->L.nc : nullptr;
+        ca.offs = ca.outl ? ca.outl + p->L.nc : nullptr;
+        ca.out = d_out;
+        ca.out_cap = cap;
+        ca.result = p->d_rb->result;
+        ca.err = &p->d_rb->err;
+        ca.outlier_cap = p->outlier_cap;
+        timing_mark(p, st, true, "encode");
+        eblc_status_t s = cuda_status(launch_chunked_encode(ca, p->num_sms, st), "chunked encode launch");
+        timing_mark(p, st, false, nullptr);
+        if (s != EBLC_OK) return s;
+        FinishArgs fa{p->d_rb->result, &p->d_rb->err, &p->d_rb->epoch, d_user, p->status, 2 * p->ntiles};
+        if ((s = cuda_status(launch_finish(fa, st), "finish launch")) != EBLC_OK) return s;
+        if (!d_user)
+            s = cuda_status(cudaMemcpyAsync(p->h_rb, p->d_rb, sizeof(Readback), cudaMemcpyDeviceToHost, st),
+                            "readback");
+        if (call_events) timing_end(p, st);
+        return s;
+    }
     EncodeArgs ea{};
     ea.in = d_in;
     ea.n = p->n;
@@ -366,6 +410,21 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
     return s;
 }
 
+// The plan's decoder: the block codec or the chunked one.
+cudaError_t launch_plan_decode(const eblc_plan_s *p, const DecodeArgs &da, cudaStream_t st) {
+    if (!p->chunked_m) return launch_decode(da, p->num_sms, st);
+    ChunkedDecArgs ca{};
+    ca.in = da.in;
+    ca.n = da.n;
+    ca.m = p->chunked_m;
+    ca.W = da.W;
+    ca.mo = da.m;
+    ca.step = da.step;
+    ca.out = da.out;
+    ca.err = da.err;
+    return launch_chunked_decode(ca, p->num_sms, st);
+}
+
 eblc_status_t finish_compress(eblc_plan_s *p, size_t *compressed_bytes, void *h_sidecar) {
     const Readback &rb = *p->h_rb;
     const uint32_t err = (uint32_t)rb.result[7];
@@ -375,9 +434,10 @@ eblc_status_t finish_compress(eblc_plan_s *p, size_t *compressed_bytes, void *h_
         eblc_sidecar_t sc{};
         sc.magic = kMagic;
         sc.version = (uint16_t)kVersion;
-        sc.flags = (uint16_t)((p->abs_mode ? kFlagAbs : 0) | (p->nd ? kFlagLorenzoNd : 0));
+        sc.flags = (uint16_t)((p->abs_mode ? kFlagAbs : 0) | (p->nd ? kFlagLorenzoNd : 0) |
+                              (p->chunked_m ? kFlagChunked : 0));
         sc.block = p->block;
-        sc.chunk = kChunk;
+        sc.chunk = p->chunked_m ? p->chunked_m : kChunk;
         sc.n = p->n;
         sc.total_bytes = total;
         sc.payload_words = rb.result[0];
@@ -404,10 +464,12 @@ struct StreamInfo {
 // Validate the sidecar (or the header it was rebuilt from) against the plan.
 eblc_status_t check_stream(const eblc_plan_s *p, const eblc_sidecar_t &sc, size_t compressed_bytes,
                            StreamInfo *info) {
-    if (sc.magic != kMagic || sc.version != kVersion || sc.chunk != kChunk) return EBLC_CORRUPT;
+    if (sc.magic != kMagic || sc.version != kVersion) return EBLC_CORRUPT;
+    if (sc.chunk != (p->chunked_m ? p->chunked_m : kChunk)) return p->chunked_m ? EBLC_INVALID_ARG : EBLC_CORRUPT;
+    if (((sc.flags & kFlagChunked) != 0) != (p->chunked_m != 0)) return EBLC_INVALID_ARG;  // the plan's codec
     if (sc.n != p->n || sc.block != p->block) return EBLC_INVALID_ARG;
     if (((sc.flags & kFlagLorenzoNd) != 0) != (p->nd != 0)) return EBLC_INVALID_ARG;  // the plan's predictor
-    if (sc.payload_words > sc.n || sc.n_outliers > sc.n) return EBLC_CORRUPT;
+    if (sc.payload_words > sc.n + 32 * p->L.nc || sc.n_outliers > sc.n) return EBLC_CORRUPT;
     const uint64_t total = p->L.record_off + 4 * (sc.payload_words + 2 * sc.n_outliers);
     if (total != sc.total_bytes || compressed_bytes < total) return EBLC_CORRUPT;
     info->total = total;
@@ -499,6 +561,18 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
         return s;
     }
     p->n = n;
+    if (p->opt_chunk_bytes && !p->opt_chunked) {  // chunk= belongs to codec=chunked
+        delete p;
+        return EBLC_INVALID_ARG;
+    }
+    if (p->opt_chunked) {
+        if (p->nd) {  // one codec per plan
+            delete p;
+            return EBLC_UNSUPPORTED;
+        }
+        p->chunked_m = (p->opt_chunk_bytes ? p->opt_chunk_bytes : 16384) / 4;
+        p->block = 0;  // no blocks: the stream has no width bytes
+    }
     if (p->nd) {  // multi-dimensional Lorenzo: rank 2 or 3, dims multiples of the brick, block 64 or 256
         const int r = rank;
         const uint64_t be = (r == 3) ? 16 : 64;
@@ -516,8 +590,14 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
         p->dims[2] = (uint64_t)dims[r - 1];
     }
     p->outlier_cap = std::min<uint64_t>(p->outlier_cap, n);
-    p->L = stream_layout(n, p->block);
-    p->max_bytes = p->L.record_off + 4 * (n + 2 * p->outlier_cap);
+    if (p->chunked_m) {
+        p->L = chunked_layout(n, p->chunked_m);
+        // per chunk: a head word and at most its codes padded to 32, then the outliers
+        p->max_bytes = p->L.record_off + 4 * (p->L.nc + n + 31 * p->L.nc + 2 * p->outlier_cap);
+    } else {
+        p->L = stream_layout(n, p->block);
+        p->max_bytes = p->L.record_off + 4 * (n + 2 * p->outlier_cap);
+    }
 
     if ((s = cuda_status(cudaGetDevice(&p->device), "cudaGetDevice")) != EBLC_OK) {
         delete p;
@@ -555,6 +635,14 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
             base = static_cast<uint8_t *>(p->scratch);
         }
     }
+    if (p->chunked_m && p->L.nc) {  // record slots of the chunked codec, then sizes, outlier counts, offsets
+        const uint64_t words = p->L.nc * (chunked_slot_words(p->chunked_m) + 3);
+        if ((s = cuda_status(cudaMalloc(&p->chunk_scratch, 4 * words), "cudaMalloc chunk scratch")) != EBLC_OK) {
+            p->chunk_scratch = nullptr;
+            destroy(p);
+            return s;
+        }
+    }
     if ((s = cuda_status(cudaMemset(p->scratch, 0, off), "cudaMemset")) != EBLC_OK ||
         (s = cuda_status(cudaMallocHost(&p->h_rb, sizeof(Readback)), "cudaMallocHost")) != EBLC_OK ||
         (s = cuda_status(cudaMallocHost(&p->h_err, 256), "cudaMallocHost")) != EBLC_OK) {
@@ -582,7 +670,7 @@ EBLC_API eblc_status_t eblc_plan_get_limits(eblc_plan_t p, eblc_limits_t *out) {
     std::memset(out, 0, sizeof(*out));
     out->n = p->n;
     out->block = p->block;
-    out->chunk = kChunk;
+    out->chunk = p->chunked_m ? p->chunked_m : kChunk;
     out->max_compressed_bytes = p->max_bytes;
     out->payload_alignment = kPayloadAlignment;
     out->sidecar_bytes = kSidecarBytes;
@@ -643,6 +731,7 @@ EBLC_API eblc_status_t eblc_compress_async(eblc_plan_t p, const eblc_execution_t
     if (!aligned16(d_out) || (d_in && !aligned16(d_in)) || (reinterpret_cast<uintptr_t>(d_result) & 7u))
         return EBLC_INVALID_ARG;
     if (out_capacity < p->L.record_off) return EBLC_CAPACITY;
+    if (p->chunked_m) return EBLC_UNSUPPORTED;  // the chunked codec has its synchronous calls only
     DeviceGuard g(p->device);
     if (!g.ok) return EBLC_CUDA_ERROR;
     cudaStream_t st = static_cast<cudaStream_t>(exec->stream);
@@ -681,6 +770,7 @@ EBLC_API eblc_status_t eblc_compress_range(eblc_plan_t p, const eblc_execution_t
     if (exec->kind == EBLC_EXECUTION_HIP || exec->kind == EBLC_EXECUTION_HOST) return EBLC_UNSUPPORTED;
     if (exec->kind != EBLC_EXECUTION_CUDA) return EBLC_INVALID_ARG;
     if (p->abs_mode) return EBLC_INVALID_ARG;  // a value range only matters for a relative bound
+    if (p->chunked_m) return EBLC_UNSUPPORTED;
     if (!d_out || (p->n && !d_in)) return EBLC_INVALID_ARG;
     if (!aligned16(d_out) || (d_in && !aligned16(d_in)) || (reinterpret_cast<uintptr_t>(d_range) & 3u))
         return EBLC_INVALID_ARG;
@@ -742,7 +832,7 @@ EBLC_API eblc_status_t eblc_decompress(eblc_plan_t p, const eblc_execution_t *ex
         da.out = d_out;
         timing_begin(p, st);
         timing_mark(p, st, true, "decode");
-        s = cuda_status(launch_decode(da, p->num_sms, st), "decode launch");
+        s = cuda_status(launch_plan_decode(p, da, st), "decode launch");
         timing_mark(p, st, false, nullptr);
         timing_end(p, st);
         return s;
@@ -757,7 +847,7 @@ EBLC_API eblc_status_t eblc_decompress(eblc_plan_t p, const eblc_execution_t *ex
         EBLC_OK)
         return s;
     timing_mark(p, st, true, "decode");
-    s = cuda_status(launch_decode(da, p->num_sms, st), "decode launch");
+    s = cuda_status(launch_plan_decode(p, da, st), "decode launch");
     timing_mark(p, st, false, nullptr);
     if (s != EBLC_OK) return s;
     if (p->n && (s = cuda_status(cudaMemcpyAsync(d_out, p->stage_in, 4 * p->n, cudaMemcpyDeviceToHost, st),

@@ -111,9 +111,11 @@ typedef struct {
     uint32_t magic;         /* 0x434C4245 ("EBLC")                   */
     uint16_t version;       /* stream version (1)                    */
     uint16_t flags;         /* bit0: absolute bound; bit1: 2-D / 3-D
-                               Lorenzo (lorenzo=nd)                  */
-    uint32_t block;         /* B                                     */
-    uint32_t chunk;         /* 4096                                  */
+                               Lorenzo (lorenzo=nd); bit2: chunked
+                               codec (codec=chunked)                 */
+    uint32_t block;         /* B (0 for the chunked codec)           */
+    uint32_t chunk;         /* elements per chunk: 4096, or the
+                               chunked codec's 1024 / 2048 / 4096    */
     uint64_t n;             /* elements                              */
     uint64_t total_bytes;   /* stream length                         */
     uint64_t payload_words; /* W                                     */
@@ -164,6 +166,16 @@ EBLC_API const char *eblc_status_string(eblc_status_t status);
  *                    bricks of 64x64 or 16x16x16 elements take the place of
  *                    the 4096-element chunks.  Otherwise EBLC_UNSUPPORTED.
  *                    Default lorenzo=1d: the data coded as one flat sequence
+ *   codec=chunked    the chunk-cooperative codec instead of the block codec:
+ *                    per chunk of `chunk` bytes of input, the quantization
+ *                    codes' first differences (zigzag form), bit-shuffled
+ *                    (32 bit planes per group of 32 codes) and zero-eliminated
+ *                    (a bitmap of the nonzero words, then those words), or
+ *                    kept verbatim when that is not smaller.  Not with
+ *                    lorenzo=nd; eblc_compress_async and eblc_compress_range
+ *                    return EBLC_UNSUPPORTED for such plans.  ("Pipeline
+ *                    specialization internals", Chunk-cooperative path.)
+ *   chunk=<bytes>    4096 | 8192 | 16384 (default 16384), with codec=chunked
  *   timing=1         record per-kernel device times (eblc_plan_kernel_times)
  *   wait_ms=<t>      limit of device-side waits in milliseconds (default 2000)
  *   stall_tile=<t>   test hook: tile t of one compress call never publishes
