@@ -47,31 +47,30 @@ namespace {
 
 constexpr int kNW = 8;                    // compute warps
 constexpr int kS = 3;                     // input stages
-constexpr int kD = 8;                     // tile slots: at most kD - 1 tiles computed but not finished
+#ifndef EBLC_ENC_SLOTS
+#define EBLC_ENC_SLOTS 16
+#endif
+constexpr int kD = EBLC_ENC_SLOTS;        // tile slots: at most kD - 1 tiles computed but not finished
 constexpr int kLookbackWarps = 3;
 constexpr int kProducerWarp = kNW + kLookbackWarps;
 constexpr int kThreads = (kNW + kLookbackWarps + 1) * 32;
 constexpr int kWindow = 10;               // look-back rows of 32 status words per round trip
-#ifndef EBLC_ENC_PREFETCH
-#define EBLC_ENC_PREFETCH 0
-#endif
-constexpr int kPrefetch = EBLC_ENC_PREFETCH;  // tiles of this CTA fetched into L2 ahead of their bulk copy
-#ifndef EBLC_ENC_LDGSTS
-#define EBLC_ENC_LDGSTS 0
-#endif
-// 1-D tiles: 1 = every producer lane moves 32 x 16 bytes with cp.async (through
-// L1), 0 = one bulk copy of the whole tile.
-constexpr int kLdgsts = EBLC_ENC_LDGSTS;
 constexpr uint32_t kRing = 1536;          // packed words a compute warp can hold (3 worst-case tiles)
 constexpr uint32_t kWarpMax = kChunk / kNW;  // most words a warp packs for one tile
-static_assert(kRing >= 3 * kWarpMax, "one pending part must always leave room for the next");
+// A compute warp short of ring room waits only for the write-out of its own
+// earlier tiles, whose look-backs wait only for lower tiles: no cycle.  The
+// ring holds several typical tiles per warp so the compute warps can run
+// ahead of the look-back (kRing >= 2 kWarpMax lets a worst-case tile follow a
+// pending one without waiting).
+static_assert(kRing >= 2 * kWarpMax, "a worst-case part must fit beside a pending one");
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint64_t kInclBit = 1ull << 63;
 
 struct __align__(128) EncSmem {
     float in[kS][kChunk];                 // input ring (bulk-copy destination)
     uint32_t ring[kNW][kRing];            // per compute warp: packed words awaiting their prefix
-    uint32_t omask[kD][kNW][32];          // per slot, warp, lane: outlier bits
+    uint16_t omask[kD][kNW][32];          // per slot, warp, lane: outlier bits (2 warp-tiles x 8);
+                                          // for 2-D / 3-D bricks the slot's 4096-bit C-order bitmap
     uint8_t width[kD][kChunk / 32];       // per slot: width bytes of the tile's blocks
     uint32_t totals[kD][kNW][2];          // per slot, warp: payload words, outliers
     uint32_t ringpos[kD][kNW];            // per slot, warp: ring offset of the packed words
@@ -85,6 +84,9 @@ struct __align__(128) EncSmem {
     uint64_t written[kD];                 // completes once per use of the slot: its tile is written out
     Bound bound;
 };
+
+// Two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA.
+static_assert(sizeof(EncSmem) <= 233472 / 2 - 1024, "two encoder CTAs must fit on an SM");
 
 // Look-back status word: bits 0..31 record words + 1 (never 0 once
 // published), bits 32..62 outliers, bit 63 set for an inclusive prefix.
@@ -595,7 +597,7 @@ __device__ __forceinline__ void compute_tile_nd(EncSmem &sm, const Bound &bd, in
     constexpr int RX = (ND == 3 && LPB == 8) ? 4 : 8;  // codes per row of a lane
     const int g = ln / LPB, r = ln % LPB;
     uint32_t wo = 0, outl = 0;
-    uint32_t *bitmap = &sm.omask[q][0][0];  // outliers of the tile, in brick C order (4096 bits)
+    uint32_t *bitmap = reinterpret_cast<uint32_t *>(&sm.omask[q][0][0]);  // brick C order, 4096 bits
 #pragma unroll 1
     for (int k = 0; k < kWPW; ++k) {
         const int wt = cw * kWPW + k;
@@ -701,7 +703,7 @@ __device__ void compute_warp(EncSmem &sm, const EncodeArgs &a, int cw, int ln) {
                 compute_tile<V, LPB>(sm, bd, s, q, valid, cw, ln, ring + start, words, omask);
             }
             outl = __reduce_add_sync(kFull, __popc(omask));
-            sm.omask[q][cw][ln] = omask;
+            sm.omask[q][cw][ln] = (uint16_t)omask;  // kWPW * V = 16 bits
         }
         __syncwarp();
         if (ln == 0) {
@@ -910,7 +912,7 @@ __device__ __forceinline__ void write_tile_nd(EncSmem &sm, const EncodeArgs &a, 
         for (uint32_t j = ln; j < lim; j += 32) st_cs_u32(dst + j, src[j]);
     }
     if (MT != 0u) {
-        uint32_t *bm = &sm.omask[q][0][0] + 4 * ln;
+        uint32_t *bm = reinterpret_cast<uint32_t *>(&sm.omask[q][0][0]) + 4 * ln;
         const uint4 b4 = *reinterpret_cast<const uint4 *>(bm);
         const uint32_t cnt = __popc(b4.x) + __popc(b4.y) + __popc(b4.z) + __popc(b4.w);
         uint32_t incl = cnt;
@@ -1114,14 +1116,10 @@ __device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
 
         uint32_t exR = 0, exM = 0;
         if (tile != 0) {  // the aggregate is already published by the compute warps
-            // Start once this CTA has also computed its next tile: by then the
-            // other CTAs have almost always published this tile's predecessors
-            // of the same wave, so the look-back rarely has to wait.  This wait
-            // cannot close a cycle: a compute warp at iteration i + 1 never
-            // needs tile i written out, because with a single pending part of
-            // at most kWarpMax words a ring of 3 * kWarpMax words always has
-            // kWarpMax contiguous free words.
-            if (!mbar_wait(&sm.computed[(i + 1) % kD], ((i + 1) / kD) & 1, a.wait_ns, a.err)) return;
+            // The look-back waits only for aggregates of lower tiles, which
+            // their CTAs publish as soon as they have computed them; the compute
+            // warps meanwhile run up to kD - 2 tiles ahead of the write-out, so
+            // a wave's tiles are rarely still missing by the time it is read.
             look_back(a, sm.st_cur, tile, -1, pack_status(0, 0, true), ln, exR, exM);
             if (ln == 0 && publish) st_relaxed_gpu(&sm.st_cur[tile], pack_status(exR + Rt, exM + MT, true));
         }
@@ -1160,42 +1158,9 @@ __device__ void lookback_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
 // launched cooperatively (all CTAs resident at once), so every tile a
 // look-back waits for belongs to a running CTA that reaches it without
 // waiting on anything later: the look-back cannot deadlock.
-// L2 prefetch of this CTA's tile of iteration i (a whole tile, or the part of
-// the last tile that bulk copies read).
-__device__ __forceinline__ void prefetch_tile(const EncodeArgs &a, const Layout &L, uint32_t i) {
-    const uint64_t t = (uint64_t)blockIdx.x + (uint64_t)i * gridDim.x;
-    if (t >= L.nc) return;
-    const uint64_t e0 = t * kChunk;
-    const uint32_t bytes = (uint32_t)min((uint64_t)kChunk, a.n - e0) * 4u & ~15u;
-    if (bytes) prefetch_l2(a.in + e0, bytes);
-}
-
-// The same for a brick of a multi-dimensional array (its tensor-map box).
-template <int ND>
-__device__ __forceinline__ void prefetch_brick(const EncodeArgs &a, const Layout &L, uint32_t i) {
-    const uint64_t t = (uint64_t)blockIdx.x + (uint64_t)i * gridDim.x;
-    if (t >= L.nc) return;
-    int z, y, x;
-    brick_origin(t, ND, a.dims, z, y, x);
-    if constexpr (ND == 3)
-        tensor_prefetch_3d(&a.tmap, x, y, z);
-    else
-        tensor_prefetch_2d(&a.tmap, x, y);
-}
-
 template <int ND>
 __device__ void producer_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L, int ln) {
-    constexpr bool kLanes = (ND == 0 && kLdgsts != 0);  // all 32 lanes copy
-    if (!kLanes && ln != 0) return;
-    // The shared-memory stages alone keep too few bytes in flight to cover
-    // DRAM latency under load; the tiles kPrefetch iterations ahead are
-    // fetched into L2 early, so the stage copies mostly hit L2.
-    for (uint32_t j = 1; ln == 0 && j <= (uint32_t)kPrefetch; ++j) {
-        if constexpr (ND != 0)
-            prefetch_brick<ND>(a, L, j);
-        else
-            prefetch_tile(a, L, j);
-    }
+    if (ln != 0) return;
     // Tensor copies want a 128-byte aligned shared destination; the stages are
     // laid out for that, and a launch where it does not hold reports an error
     // and ends (every tile marked absent) instead of issuing the copy.
@@ -1205,26 +1170,14 @@ __device__ void producer_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
     for (;; ++i) {
         const int s = i % kS;
         if (i >= kS && !mbar_wait(&sm.empty[s], ((i / kS) - 1) & 1, a.wait_ns, a.err)) break;
-        if (i >= 1 && kPrefetch > 0 && ln == 0) {
-            if constexpr (ND != 0)
-                prefetch_brick<ND>(a, L, i + kPrefetch);
-            else
-                prefetch_tile(a, L, i + kPrefetch);
-        }
         const uint64_t t = (uint64_t)blockIdx.x + (uint64_t)i * gridDim.x;
         if (t >= L.nc || !tensor_ok) {
-            if (ln == 0) sm.tile_id[s] = -1;
-            if constexpr (kLanes) {
-                __syncwarp();
-                mbar_arrive(&sm.full[s]);  // 32 lanes ...
-                if (ln == 0) mbar_arrive(&sm.full[s]);  // ... + 1: the stage's expected count
-            } else {
-                mbar_arrive(&sm.full[s]);
-            }
+            sm.tile_id[s] = -1;
+            mbar_arrive(&sm.full[s]);
             ++i;
             break;
         }
-        if (ln == 0) sm.tile_id[s] = (int32_t)t;
+        sm.tile_id[s] = (int32_t)t;
         if constexpr (ND != 0) {  // a whole brick by one tensor copy, C order in the stage
             int z, y, x;
             brick_origin(t, ND, a.dims, z, y, x);
@@ -1238,20 +1191,9 @@ __device__ void producer_warp(EncSmem &sm, const EncodeArgs &a, const Layout &L,
         const uint64_t e0 = t * kChunk;
         const uint32_t valid = (uint32_t)min((uint64_t)kChunk, a.n - e0);
         const uint32_t bulk = (valid * 4u) & ~15u;
-        if constexpr (kLanes) {
-            // 16-byte pieces c = 32 k + lane; the ragged tail by lane 0 with
-            // plain loads, published by its ordinary arrive (count 33)
-            for (uint32_t c = ln; c < bulk / 16; c += 32) async_copy16(&sm.in[s][4 * c], a.in + e0 + 4 * c);
-            async_copy_arrive(&sm.full[s]);
-            if (ln == 0) {
-                for (uint32_t j = bulk / 4; j < valid; ++j) sm.in[s][j] = a.in[e0 + j];
-                mbar_arrive(&sm.full[s]);
-            }
-        } else {
-            for (uint32_t j = bulk / 4; j < valid; ++j) sm.in[s][j] = a.in[e0 + j];
-            mbar_arrive_expect_tx(&sm.full[s], bulk);
-            if (bulk) bulk_g2s(sm.in[s], a.in + e0, bulk, &sm.full[s]);
-        }
+        for (uint32_t j = bulk / 4; j < valid; ++j) sm.in[s][j] = a.in[e0 + j];
+        mbar_arrive_expect_tx(&sm.full[s], bulk);
+        if (bulk) bulk_g2s(sm.in[s], a.in + e0, bulk, &sm.full[s]);
     }
     // Drain: no copy into this CTA's shared memory may still be in flight at exit.
     for (int s = 0; s < kS; ++s) {
@@ -1269,7 +1211,7 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kS; ++s) {
-            mbar_init(&sm.full[s], (ND == 0 && kLdgsts) ? 33 : 1);
+            mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], kNW);
         }
         for (int q = 0; q < kD; ++q) {
@@ -1281,7 +1223,7 @@ __global__ void __launch_bounds__(kThreads, 2) encode_kernel(const __grid_consta
         }
         mbar_init_fence();
         if (ND != 0)  // the outlier bitmaps of the slots start clear
-            for (int j = 0; j < kD * kNW * 32; ++j) (&sm.omask[0][0][0])[j] = 0u;
+            for (int j = 0; j < kD * kNW * 32; ++j) (&sm.omask[0][0][0])[j] = 0;
         float vmin = a.abs_mode ? 0.0f : a.range[0] + 0.0f;  // + 0: -0 reads as +0
         float vmax = a.abs_mode ? 0.0f : a.range[1] + 0.0f;
         if (!a.abs_mode && a.range_given && blockIdx.x == 0 &&

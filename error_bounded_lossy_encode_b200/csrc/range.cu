@@ -7,8 +7,7 @@
 //
 // HBM-bound: 4 bytes read per element, no writes.  Persistent grid of one
 // wave of 256-thread CTAs; each thread keeps 8 float4 loads in flight
-// (fetched with a 256-byte L2 prefetch hint), and each CTA prefetches the
-// pieces of its next sweep into L2 with bulk prefetches.
+// (fetched with a 256-byte L2 prefetch hint).
 // The array is walked from its end to its start so the lowest addresses are
 // the last read and are still in L2 when the encoder starts at tile 0.
 #include "common.cuh"
@@ -43,15 +42,6 @@ __global__ void __launch_bounds__(kThreads) range_kernel(RangeArgs a) {
     const uint64_t tid = (uint64_t)blockIdx.x * kThreads + threadIdx.x;
 
     for (uint64_t base = 0; base < n4; base += stride * kUnroll) {
-        // The next sweep's 4 KB pieces of this CTA (one per unroll slot) are
-        // fetched into L2 now, so its loads mostly hit L2.
-        if (threadIdx.x < kUnroll) {
-            const uint64_t i0 = base + stride * kUnroll + threadIdx.x * stride + (uint64_t)blockIdx.x * kThreads;
-            if (i0 < n4) {
-                const uint64_t last = min(i0 + kThreads, n4) - 1;  // pieces run downwards from n4 - 1 - i0
-                prefetch_l2(in4 + (n4 - 1 - last), (uint32_t)(last - i0 + 1) * 16u);
-            }
-        }
         float4 v[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
