@@ -36,10 +36,6 @@ constexpr int kThreads = (kNW + 1) * 32;
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint32_t kStagedOutliers = 1024;                 // outliers staged with the payload
 constexpr uint32_t kRecWords = kChunk + 2 * kStagedOutliers + 4 + 16;  // + alignment + over-read slack
-#ifndef EBLC_DEC_PREFETCH
-#define EBLC_DEC_PREFETCH 0
-#endif
-constexpr int kPrefetch = EBLC_DEC_PREFETCH;  // chunks of this CTA whose records are fetched into L2 ahead
 
 struct __align__(128) DecSmem {
     uint32_t rec[kS][kRecWords];
@@ -388,25 +384,26 @@ __device__ void producer_warp(DecSmem &sm, const DecodeArgs &a, int ln) {
     const uint64_t R = a.W + 2 * a.m;
     const uint32_t K = kChunk / a.block;  // blocks per chunk
     const uint64_t total16 = a.total & ~uint64_t(15);
-    // L2 prefetch of the record of this CTA's chunk of iteration j (its
-    // extent from the chunk index, clamped to the stream; only a hint, so a
-    // corrupt index costs nothing but the prefetch).
-    auto prefetch_record = [&](uint32_t j) {
-        const uint64_t tp = (uint64_t)blockIdx.x + (uint64_t)j * gridDim.x;
-        if (tp >= L.nc) return;
-        const uint64_t r0 = *reinterpret_cast<const uint32_t *>(a.in + L.index_off + 8 * tp);
-        const uint64_t r1 = (tp + 1 < L.nc) ? *reinterpret_cast<const uint32_t *>(a.in + L.index_off + 8 * (tp + 1)) : R;
-        const uint64_t b0 = (L.record_off + 4 * r0) & ~uint64_t(15);
-        const uint64_t b1 = min((L.record_off + 4 * r1 + 15) & ~uint64_t(15), total16);
-        if (r1 > r0 && b1 > b0 && b1 - b0 <= 4ull * kRecWords) prefetch_l2(a.in + b0, (uint32_t)(b1 - b0));
+    // The chunk index entries of a chunk and of the one after it, for the
+    // chunk of iteration i; those of iteration i + 1 are loaded one iteration
+    // ahead, so a stage fill waits for its bulk copy only, not for an index
+    // read before it.
+    auto index_pair = [&](uint64_t t, uint2 &ent, uint2 &nx) {
+        ent = make_uint2(0u, 0u);
+        nx = make_uint2((uint32_t)R, (uint32_t)a.m);
+        if (t < L.nc) ent = *reinterpret_cast<const uint2 *>(a.in + L.index_off + 8 * t);
+        if (t + 1 < L.nc) nx = *reinterpret_cast<const uint2 *>(a.in + L.index_off + 8 * (t + 1));
     };
-    for (uint32_t j = 1; j <= (uint32_t)kPrefetch; ++j) prefetch_record(j);
+    uint2 ent_ahead, nx_ahead;
+    index_pair(blockIdx.x, ent_ahead, nx_ahead);
     uint32_t i = 0;
     for (;; ++i) {
         const int s = i % kS;
-        if (i >= kS && !mbar_wait(&sm.empty[s], ((i / kS) - 1) & 1, a.wait_ns, a.err)) break;
-        if (i >= 1 && kPrefetch > 0) prefetch_record(i + kPrefetch);
         const uint64_t t = (uint64_t)blockIdx.x + (uint64_t)i * gridDim.x;
+        const uint2 ent = ent_ahead;
+        uint64_t rec_next = (t + 1 < L.nc) ? nx_ahead.x : R, bef_next = (t + 1 < L.nc) ? nx_ahead.y : a.m;
+        index_pair(t + gridDim.x, ent_ahead, nx_ahead);  // next iteration's entries, in flight meanwhile
+        if (i >= kS && !mbar_wait(&sm.empty[s], ((i / kS) - 1) & 1, a.wait_ns, a.err)) break;
         if (t >= L.nc) {
             sm.info[s][0] = (uint32_t)-1;
             mbar_arrive(&sm.full[s]);
@@ -415,13 +412,6 @@ __device__ void producer_warp(DecSmem &sm, const DecodeArgs &a, int ln) {
         }
         const uint64_t e0 = t * kChunk;
         const uint32_t valid = (uint32_t)min((uint64_t)kChunk, a.n - e0);
-        const uint2 ent = *reinterpret_cast<const uint2 *>(a.in + L.index_off + 8 * t);
-        uint64_t rec_next = R, bef_next = a.m;
-        if (t + 1 < L.nc) {
-            const uint2 nx = *reinterpret_cast<const uint2 *>(a.in + L.index_off + 8 * (t + 1));
-            rec_next = nx.x;
-            bef_next = nx.y;
-        }
         uint32_t corrupt = 0, PW = 0, mt = 0;
         if (rec_next < ent.x || bef_next < ent.y || rec_next > R || bef_next > a.m) {
             corrupt = 1;

@@ -51,7 +51,10 @@ constexpr int kS = 3;                     // input stages
 #define EBLC_ENC_SLOTS 16
 #endif
 constexpr int kD = EBLC_ENC_SLOTS;        // tile slots: at most kD - 1 tiles computed but not finished
-constexpr int kLookbackWarps = 3;
+#ifndef EBLC_ENC_LB
+#define EBLC_ENC_LB 3
+#endif
+constexpr int kLookbackWarps = EBLC_ENC_LB;  // look-back and write-out warps
 constexpr int kProducerWarp = kNW + kLookbackWarps;
 constexpr int kThreads = (kNW + kLookbackWarps + 1) * 32;
 constexpr int kWindow = 10;               // look-back rows of 32 status words per round trip
