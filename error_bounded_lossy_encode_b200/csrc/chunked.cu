@@ -5,20 +5,23 @@
 // File Reference", launchNvrtcChunkFusedEncode: each chunk's coded form in a
 // scratch slot with its size, then the cross-chunk scan/pack tail).
 //
-//   chunk_encode  one CTA per chunk (grid-stride): the linear quantizer and
+//   chunk_encode  one CTA per chunk (grid-stride), each warp a contiguous run
+//                 of 32-code groups in registers: the linear quantizer and
 //                 the outlier test, first differences reset at the chunk start
-//                 in zigzag form, the 32-plane bit transpose of every group of
-//                 32 codes by warp ballots, zero elimination (a bitmap of the
-//                 nonzero words by ballots, the nonzero words compacted by a
-//                 block scan) or the shuffled words verbatim when that is not
-//                 smaller, then the chunk's outliers in ascending order; the
-//                 record goes to the chunk's scratch slot, its size to sizes[].
+//                 in zigzag form, the 32 x 32 bit transpose of every group
+//                 (lane b gets bit plane b) by a shuffle butterfly, zero
+//                 elimination (a bitmap of the nonzero words by ballots, the
+//                 nonzero words compacted warp by warp after one block scan)
+//                 or the shuffled words verbatim when that is not smaller,
+//                 then the chunk's outliers in ascending order; the record
+//                 goes to the chunk's scratch slot, its size to sizes[].
 //   chunk_scan    one CTA: exclusive scan of the record sizes and outlier
 //                 counts -> chunk index, header and result block.
 //   chunk_gather  records from scratch to their place in the stream.
 //   chunk_decode  one CTA per chunk: zero elimination undone (ranks by
-//                 popcounts), the inverse bit transpose by ballots, zigzag
-//                 undone, a block-wide prefix sum, dequantization, outliers.
+//                 popcounts), the inverse transpose, zigzag undone and the
+//                 prefix sum in each warp's registers, one block scan of the
+//                 warps' totals, dequantization, outliers.
 // No inter-CTA waits anywhere: the scan is its own launch.
 #include "common.cuh"
 #include "kernels.h"
@@ -29,9 +32,24 @@ namespace {
 constexpr int kCT = 256;                  // threads per CTA
 constexpr int kCW = kCT / 32;
 constexpr uint32_t kFull = 0xffffffffu;
-constexpr uint32_t kMaxM = 4096;          // largest chunk, elements
 
 __device__ __forceinline__ uint32_t zz(int32_t d) { return ((uint32_t)d << 1) ^ (uint32_t)(d >> 31); }
+
+// 32 x 32 bit-matrix transpose across the warp: on entry lane r holds row r
+// (bit c = element (r, c)), on return lane c holds column c (bit r = element
+// (r, c)).  Five butterfly stages, each swapping the off-diagonal j x j
+// blocks between lanes r and r ^ j with one shuffle.
+__device__ __forceinline__ uint32_t transpose32(uint32_t w, int ln) {
+    const uint32_t masks[5] = {0x0000ffffu, 0x00ff00ffu, 0x0f0f0f0fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const int j = 16 >> k;
+        const uint32_t m = masks[k];
+        const uint32_t p = __shfl_xor_sync(kFull, w, j);
+        w = (ln & j) ? ((w & ~m) | ((p >> j) & m)) : ((w & m) | ((p & m) << j));
+    }
+    return w;
+}
 __device__ __forceinline__ int32_t unzz(uint32_t z) { return (int32_t)((z >> 1) ^ (0u - (z & 1u))); }
 
 // Exclusive block-wide prefix of v (every thread of the CTA calls it);
@@ -58,106 +76,128 @@ __device__ __forceinline__ uint32_t block_excl(uint32_t v, uint32_t *tmp, uint32
     return before + incl - v;
 }
 
-struct __align__(16) EncShared {
-    int32_t q[kMaxM];
-    uint32_t sw[kMaxM];       // shuffled words, plane-major
-    uint32_t oflag[kMaxM / 32];
-    uint32_t tmp[kCW];
-};
+// Position in shared memory of word k of a chunk's shuffled words (k =
+// plane * G + group, G groups of 32 codes).  For a full chunk G is 32, 64 or
+// 128 and word k sits at k ^ plane: the column of one group (one word per
+// plane, lanes 0..31) and a run of 32 consecutive words of one plane both
+// fall in 32 distinct banks.  A ragged last chunk keeps the plain order.
+__device__ __forceinline__ uint32_t phys(uint32_t k, int lg) { return lg ? (k ^ ((k >> lg) & 31u)) : k; }
 
+// Quantized code of x and its outlier test ("Pipeline specialization
+// internals", Quantization: fp32 filter with thresholds from the bound,
+// fp64 test in the band between them).
+__device__ __forceinline__ int32_t quant(const Bound &bd, float x, bool &o) {
+    const float y = __fmul_rn(x, bd.inv2eb);
+    const int32_t qq = (fabsf(y) < 0x1p30f) ? __float2int_rn(y) : 0;
+    const float xr = __fmul_rn(__int2float_rn(qq), bd.step);
+    const float d = fabsf(__fsub_rn(x, xr));
+    o = d > bd.t_out;
+    if (!o && !(d <= bd.t_in)) {
+        const bool finite = fabsf(x) < __int_as_float(0x7f800000);
+        o = !finite || !(fabs(__dsub_rn((double)x, (double)xr)) <= bd.eb);
+    }
+    return qq;
+}
+
+// Dynamic shared memory of the encoder for chunks of m elements: the
+// shuffled words, the outlier flag words, the scan's warp totals.
+__host__ __device__ constexpr size_t enc_smem_bytes(uint32_t m) { return 4ull * (m + m / 32 + kCW); }
+
+// PER = m / kCT.  Warp w owns the PER groups of 32 codes starting at code
+// 32 PER w of the chunk and keeps them in registers from the load to the
+// bit transpose; the input of the CTA's next chunk is loaded as soon as the
+// current chunk's codes are formed, so its latency overlaps the rest.
+template <int PER>
 __global__ void __launch_bounds__(kCT) chunk_encode(const ChunkedArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    EncShared &sm = *reinterpret_cast<EncShared *>(smem_raw);
+    uint32_t *const sw = reinterpret_cast<uint32_t *>(smem_raw);
+    uint32_t *const oflag = sw + a.m;
+    uint32_t *const tmp = oflag + a.m / 32;
     const int t = threadIdx.x, ln = t % 32, w = t / 32;
+    const int lg_full = 31 - __clz(a.m / 32);
     __shared__ Bound bd;
     if (t == 0) {
         const float vmin = a.abs_mode ? 0.0f : a.range[0], vmax = a.abs_mode ? 0.0f : a.range[1];
         bd = resolve_bound(a.abs_mode, a.bound, vmin, vmax);
     }
+    const uint32_t first = (uint32_t)(32 * PER * w);  // the warp's first code in its chunk
+    float xv[PER], xp = 0.0f;
+    auto load = [&](uint64_t c) {
+        const uint64_t e0 = c * a.m;
+        const uint32_t cnt = (c < a.nc) ? (uint32_t)min((uint64_t)a.m, a.n - e0) : 0u;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const uint32_t j = first + 32 * i + ln;
+            xv[i] = (j < cnt) ? __ldcs(a.in + e0 + j) : 0.0f;
+        }
+        // the code before the warp's first one (its difference), re-quantized here
+        xp = (ln == 0 && first > 0 && first <= cnt) ? a.in[e0 + first - 1] : 0.0f;
+    };
+    load(blockIdx.x);
     __syncthreads();
     for (uint64_t c = blockIdx.x; c < a.nc; c += gridDim.x) {
         const uint64_t e0 = c * a.m;
         const uint32_t cnt = (uint32_t)min((uint64_t)a.m, a.n - e0), mp = (cnt + 31u) & ~31u, G = mp / 32;
+        const int lg = (mp == a.m) ? lg_full : 0;
         uint32_t *rec = a.scratch + c * (uint64_t)a.slot_words;
-        for (uint32_t j = t; j < G; j += kCT) sm.oflag[j] = 0u;
-        __syncthreads();
-        // Quant: codes and outlier flags (fp32 filter, fp64 test in the band)
-        for (uint32_t j = t; j < mp; j += kCT) {
-            int32_t qq = 0;
-            if (j < cnt) {
-                const float x = a.in[e0 + j];
-                const float y = __fmul_rn(x, bd.inv2eb);
-                qq = (fabsf(y) < 0x1p30f) ? __float2int_rn(y) : 0;
-                const float xr = __fmul_rn(__int2float_rn(qq), bd.step);
-                const float d = fabsf(__fsub_rn(x, xr));
-                bool o = d > bd.t_out;
-                if (!o && !(d <= bd.t_in)) {
-                    const bool finite = fabsf(x) < __int_as_float(0x7f800000);
-                    o = !finite || !(fabs(__dsub_rn((double)x, (double)xr)) <= bd.eb);
-                }
-                if (o) atomicOr(&sm.oflag[j >> 5], 1u << (j & 31u));
-            }
-            sm.q[j] = qq;
-        }
-        __syncthreads();
-        // Diff (zigzag) and Bitshuffle: warp w takes groups g = w, w + 8, ...;
-        // lane l holds code 32 g + l; ballot b gives plane b's word of the group.
-        for (uint32_t g = w; g < G; g += kCW) {
-            const uint32_t j = g * 32 + ln;
-            const uint32_t d = (j < cnt) ? zz(sm.q[j] - (j ? sm.q[j - 1] : 0)) : 0u;
-            uint32_t mine = 0;
+        // Quant, Diff (zigzag, reset at the chunk start) and Bitshuffle of the
+        // warp's groups: lane l holds code 32 g + l; the transpose gives lane b
+        // plane b's word of the group.
+        bool o;
+        int32_t prev = 0;
+        if (ln == 0 && first > 0 && first <= cnt) prev = quant(bd, xp, o);
 #pragma unroll
-            for (int b = 0; b < 32; ++b) {
-                const uint32_t pb = __ballot_sync(kFull, (d >> b) & 1u);
-                if (ln == b) mine = pb;
-            }
-            sm.sw[ln * G + g] = mine;
+        for (int i = 0; i < PER; ++i) {
+            const uint32_t g = first / 32 + i, j = 32 * g + ln;
+            if (g >= G) break;  // warp-uniform
+            o = false;
+            const int32_t qq = (j < cnt) ? quant(bd, xv[i], o) : 0;
+            int32_t left = __shfl_up_sync(kFull, qq, 1);
+            if (ln == 0) left = prev;
+            prev = __shfl_sync(kFull, qq, 31);
+            const uint32_t d = (j < cnt) ? zz(qq - left) : 0u;
+            const uint32_t fw = __ballot_sync(kFull, o);
+            if (ln == 0) oflag[g] = fw;
+            sw[phys(ln * G + g, lg)] = transpose32(d, ln);
         }
+        load(c + gridDim.x);
         __syncthreads();
-        // RZE: count the nonzero words, then bitmap + compaction or verbatim
-        uint32_t nz = 0;
-        for (uint32_t k = t; k < mp; k += kCT) nz += sm.sw[k] != 0u;
-        uint32_t nnz;
-        (void)block_excl(nz, sm.tmp, &nnz);
-        const uint32_t r = G + nnz;
-        const bool raw = r >= mp;
-        const uint32_t P = raw ? mp : r;
+        // One block scan for both counts: warp w's nonzero words over its word
+        // range [k0, k1) (upper 16 bits, lane 0 only) and thread t's outliers
+        // in flag word t (lower 16 bits; G <= kCT).  Both totals are <= 4096.
+        const uint32_t per = ((G + kCW - 1) / kCW) * 32;
+        const uint32_t k0 = min(w * per, mp), k1 = min(k0 + per, mp);
+        uint32_t cntw = 0;
+        for (uint32_t k = k0 + ln; k < k1; k += 32) cntw += __popc(__ballot_sync(kFull, sw[phys(k, lg)] != 0u));
+        const uint32_t ow = (t < (int)G) ? __popc(oflag[t]) : 0u;
+        uint32_t tot;
+        const uint32_t pre = block_excl(((ln == 0 ? cntw : 0u) << 16) | ow, tmp, &tot);
+        const uint32_t nnz = tot >> 16, mc = tot & 0xffffu;
+        // RZE: bitmap + compacted nonzero words, or the words verbatim when
+        // that is not smaller
+        const bool raw = G + nnz >= mp;
+        const uint32_t P = raw ? mp : G + nnz;
         if (raw) {
-            for (uint32_t k = t; k < mp; k += kCT) rec[1 + k] = sm.sw[k];
+            for (uint32_t k = t; k < mp; k += kCT) rec[1 + k] = sw[phys(k, lg)];
         } else {
-            uint32_t base = 0;
-            for (uint32_t k0 = 0; k0 < mp; k0 += kCT) {  // rounds of one word per thread, in order
-                const uint32_t k = k0 + t;
-                const bool nzk = k < mp && sm.sw[k] != 0u;
-                const uint32_t bal = __ballot_sync(kFull, nzk);
-                if (k < mp && ln == 0) rec[1 + k / 32] = bal;  // bitmap word k / 32 (lane l: word 32 (k/32) + l)
-                uint32_t round_total;
-                const uint32_t pos = block_excl(nzk ? 1u : 0u, sm.tmp, &round_total);
-                if (nzk) rec[1 + G + base + pos] = sm.sw[k];
-                base += round_total;
+            uint32_t base = __shfl_sync(kFull, pre >> 16, 0);
+            for (uint32_t k = k0 + ln; k < k1; k += 32) {
+                const uint32_t v = sw[phys(k, lg)];
+                const uint32_t bal = __ballot_sync(kFull, v != 0u);
+                if (ln == 0) rec[1 + k / 32] = bal;  // bitmap word k / 32: bit l = word 32 (k/32) + l
+                if (v) rec[1 + G + base + __popc(bal & ((1u << ln) - 1u))] = v;
+                base += __popc(bal);
             }
         }
-        // outliers of the chunk, ascending: ranks from the flag words' popcounts
-        uint32_t oc = 0;
-        for (uint32_t j = t; j < G; j += kCT) oc += __popc(sm.oflag[j]);
-        uint32_t mc;
-        (void)block_excl(oc, sm.tmp, &mc);
-        if (mc) {
-            uint32_t obase = 0;
-            for (uint32_t j0 = 0; j0 < G; j0 += kCT) {
-                const uint32_t j = j0 + t;
-                const uint32_t fw = j < G ? sm.oflag[j] : 0u;
-                uint32_t round_total;
-                uint32_t p = obase + block_excl(__popc(fw), sm.tmp, &round_total);
-                uint32_t bits = fw;
-                while (bits) {
-                    const uint32_t e = j * 32 + (uint32_t)(__ffs(bits) - 1);
-                    bits &= bits - 1u;
-                    rec[1 + P + p] = (uint32_t)(e0 + e);
-                    rec[1 + P + mc + p] = __float_as_uint(a.in[e0 + e]);
-                    ++p;
-                }
-                obase += round_total;
+        // outliers of the chunk, ascending: thread t writes those of flag word t
+        if (t < (int)G) {
+            uint32_t bits = oflag[t], q = pre & 0xffffu;
+            while (bits) {
+                const uint32_t e = t * 32 + (uint32_t)(__ffs(bits) - 1);
+                bits &= bits - 1u;
+                rec[1 + P + q] = (uint32_t)(e0 + e);
+                rec[1 + P + mc + q] = __float_as_uint(a.in[e0 + e]);
+                ++q;
             }
         }
         if (t == 0) {
@@ -170,48 +210,61 @@ __global__ void __launch_bounds__(kCT) chunk_encode(const ChunkedArgs a) {
 }
 
 constexpr int kScanThreads = 1024;
+constexpr int kScanWarps = kScanThreads / 32;
 
 // Exclusive scan of the record sizes and outlier counts over all chunks (one
 // CTA), the chunk index and the header of the stream, the result block.
+// Warp w takes a contiguous range of chunks, 32 at a time (coalesced): one
+// pass for the warps' totals, a scan of those, a second pass for the entries.
 __global__ void __launch_bounds__(kScanThreads) chunk_scan(const ChunkedArgs a) {
-    __shared__ unsigned long long part_r[kScanThreads / 32], part_m[kScanThreads / 32];
+    __shared__ unsigned long long part_r[kScanWarps], part_m[kScanWarps];
     const int t = threadIdx.x, ln = t % 32, w = t / 32;
-    const uint64_t per = (a.nc + kScanThreads - 1) / kScanThreads;
-    const uint64_t c0 = min(a.nc, per * t), c1 = min(a.nc, c0 + per);
+    const uint64_t steps = (a.nc + 32 * kScanWarps - 1) / (32 * kScanWarps);  // 32-chunk steps per warp
+    const uint64_t c0 = min(a.nc, (uint64_t)w * steps * 32), c1 = min(a.nc, c0 + steps * 32);
     unsigned long long sr = 0, sm_ = 0;
-    for (uint64_t c = c0; c < c1; ++c) {
+#pragma unroll 4
+    for (uint64_t c = c0 + ln; c < c1; c += 32) {
         sr += a.sizes[c];
         sm_ += a.outl[c];
     }
-    unsigned long long ir = sr, im = sm_;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned long long x = __shfl_up_sync(kFull, ir, o), y = __shfl_up_sync(kFull, im, o);
-        if (ln >= o) {
-            ir += x;
-            im += y;
-        }
+    for (int o = 16; o; o >>= 1) {
+        sr += __shfl_xor_sync(kFull, sr, o);
+        sm_ += __shfl_xor_sync(kFull, sm_, o);
     }
-    if (ln == 31) {
-        part_r[w] = ir;
-        part_m[w] = im;
+    if (ln == 0) {
+        part_r[w] = sr;
+        part_m[w] = sm_;
     }
     __syncthreads();
-    unsigned long long br = 0, bm = 0, R = 0, M = 0;
-    for (int k = 0; k < kScanThreads / 32; ++k) {
-        br += (k < w) ? part_r[k] : 0ull;
-        bm += (k < w) ? part_m[k] : 0ull;
+    unsigned long long r = 0, m = 0, R = 0, M = 0;
+    for (int k = 0; k < kScanWarps; ++k) {
+        r += (k < w) ? part_r[k] : 0ull;
+        m += (k < w) ? part_m[k] : 0ull;
         R += part_r[k];
         M += part_m[k];
     }
-    unsigned long long r = br + ir - sr, m = bm + im - sm_;
     const Layout L = chunked_layout(a.n, a.m);
     const bool idx_fits = L.record_off <= a.out_cap;
-    for (uint64_t c = c0; c < c1; ++c) {
-        a.offs[c] = (uint32_t)r;
-        if (idx_fits) *reinterpret_cast<uint2 *>(a.out + L.index_off + 8 * c) = make_uint2((uint32_t)r, (uint32_t)m);
-        r += a.sizes[c];
-        m += a.outl[c];
+    for (uint64_t cb = c0; cb < c1; cb += 32) {
+        const uint64_t c = cb + ln;
+        const uint32_t s = (c < c1) ? a.sizes[c] : 0u, q = (c < c1) ? a.outl[c] : 0u;
+        uint32_t is = s, iq = q;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(kFull, is, o), y = __shfl_up_sync(kFull, iq, o);
+            if (ln >= o) {
+                is += x;
+                iq += y;
+            }
+        }
+        const uint64_t rc = r + is - s, mcc = m + iq - q;
+        if (c < c1) {
+            a.offs[c] = (uint32_t)rc;
+            if (idx_fits) *reinterpret_cast<uint2 *>(a.out + L.index_off + 8 * c) = make_uint2((uint32_t)rc, (uint32_t)mcc);
+        }
+        r += __shfl_sync(kFull, is, 31);
+        m += __shfl_sync(kFull, iq, 31);
     }
     if (t != 0) return;
     const float vmin = a.abs_mode ? 0.0f : a.range[0], vmax = a.abs_mode ? 0.0f : a.range[1];
@@ -267,67 +320,111 @@ __global__ void __launch_bounds__(kCT) chunk_gather(const ChunkedArgs a) {
     }
 }
 
-struct __align__(16) DecShared {
-    uint32_t sw[kMaxM];
-    uint32_t q[kMaxM];
-    uint32_t rank[kMaxM / 32];  // nonzero words before each bitmap word
-    uint32_t tmp[kCW];
-    uint32_t info[4];           // P, raw, mc, record word offset
-};
+// Dynamic shared memory of the decoder for chunks of m elements: the record's
+// payload words, the shuffled words, the ranks of the bitmap words, the
+// scan's warp totals and the chunk's record facts.
+__host__ __device__ constexpr size_t dec_smem_bytes(uint32_t m) { return 4ull * (2 * m + m / 32 + kCW + 4); }
 
+// PER = m / kCT.  Warp w decodes the PER groups starting at code 32 PER w:
+// the transpose, zigzag and the prefix sum stay in its registers, and its
+// reconstructions go out as whole 128-byte lines.  Thread 0 loads the index
+// entries and the head word of the CTA's next chunk one chunk ahead; the
+// payload and the first kCT outliers of a chunk come in one round of loads.
+template <int PER>
 __global__ void __launch_bounds__(kCT) chunk_decode(const ChunkedDecArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    DecShared &sm = *reinterpret_cast<DecShared *>(smem_raw);
+    uint32_t *const pl = reinterpret_cast<uint32_t *>(smem_raw);  // payload (RZE form)
+    uint32_t *const sw = pl + a.m;
+    uint32_t *const rank = sw + a.m;
+    uint32_t *const tmp = rank + a.m / 32;
+    uint32_t *const info = tmp + kCW;  // P (0xffffffff: corrupt), raw, mc, record word offset
     const int t = threadIdx.x, ln = t % 32, w = t / 32;
+    const int lg_full = 31 - __clz(a.m / 32);
     const Layout L = chunked_layout(a.n, a.m);
     const uint32_t *recs = reinterpret_cast<const uint32_t *>(a.in + L.record_off);
     const uint64_t R = a.W + 2 * a.mo;
+    const uint32_t first = (uint32_t)(32 * PER * w);
+    // thread 0: the next chunk's index entries (its own and its successor's) and head word
+    uint64_t ex = 0, ey = 0, nx = 0, ny = 0;
+    uint32_t head = 0;
+    bool eok = false;
+    auto fetch_entries = [&](uint64_t c) {
+        if (c >= L.nc) return;
+        const uint2 e = *reinterpret_cast<const uint2 *>(a.in + L.index_off + 8 * c);
+        ex = e.x;
+        ey = e.y;
+        nx = R;
+        ny = a.mo;
+        if (c + 1 < L.nc) {
+            const uint2 e2 = *reinterpret_cast<const uint2 *>(a.in + L.index_off + 8 * (c + 1));
+            nx = e2.x;
+            ny = e2.y;
+        }
+    };
+    auto fetch_head = [&]() {
+        eok = nx >= ex + 1 && ny >= ey && nx <= R && ny <= a.mo;
+        head = eok ? recs[ex] : 0u;
+    };
+    if (t == 0) {
+        fetch_entries(blockIdx.x);
+        fetch_head();
+    }
     for (uint64_t c = blockIdx.x; c < L.nc; c += gridDim.x) {
         const uint64_t e0 = c * a.m;
         const uint32_t cnt = (uint32_t)min((uint64_t)a.m, a.n - e0), mp = (cnt + 31u) & ~31u, G = mp / 32;
+        const int lg = (mp == a.m) ? lg_full : 0;
         if (t == 0) {
-            const uint2 ent = *reinterpret_cast<const uint2 *>(a.in + L.index_off + 8 * c);
-            uint64_t nx = R, nm = a.mo;
-            if (c + 1 < L.nc) {
-                const uint2 e2 = *reinterpret_cast<const uint2 *>(a.in + L.index_off + 8 * (c + 1));
-                nx = e2.x;
-                nm = e2.y;
-            }
-            uint32_t ok = nx >= (uint64_t)ent.x + 1 && nm >= ent.y && nx <= R && nm <= a.mo;
-            uint32_t P = 0, raw = 0, mc = 0;
-            if (ok) {
-                const uint32_t head = recs[ent.x];
-                P = head & 0x7fffffffu;
-                raw = head >> 31;
-                mc = (uint32_t)(nm - ent.y);
-                ok = (uint64_t)ent.x + 1 + P + 2ull * mc == nx && (raw ? P == mp : (P >= G && P < mp));
-            }
+            uint32_t P = head & 0x7fffffffu, raw = head >> 31, mc = (uint32_t)(ny - ey);
+            const bool ok = eok && ex + 1 + P + 2ull * mc == nx && (raw ? P == mp : (P >= G && P < mp));
             if (!ok) {
                 atomicOr(a.err, kErrCorrupt);
                 P = 0xffffffffu;
             }
-            sm.info[0] = P;
-            sm.info[1] = raw;
-            sm.info[2] = mc;
-            sm.info[3] = ent.x;
+            info[0] = P;
+            info[1] = raw;
+            info[2] = mc;
+            info[3] = (uint32_t)ex;
+            fetch_entries(c + gridDim.x);
         }
         __syncthreads();
-        const uint32_t P = sm.info[0], raw = sm.info[1], mc = sm.info[2];
-        const uint32_t *pay = recs + sm.info[3] + 1;
+        const uint32_t P = info[0], raw = info[1], mc = info[2];
+        const uint32_t *pay = recs + info[3] + 1;
         if (P == 0xffffffffu) {  // corrupt record: skip the chunk
+            if (t == 0) fetch_head();
             __syncthreads();
             continue;
         }
-        if (raw) {
-            for (uint32_t k = t; k < mp; k += kCT) sm.sw[k] = pay[k];
-        } else {
-            // ranks of the bitmap words (G <= 128: one warp, four words per lane)
+        uint32_t pv[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const uint32_t k = t + i * kCT;
+            pv[i] = (k < P) ? pay[k] : 0u;
+        }
+        uint32_t oi = 0, ov = 0;
+        if (t < (int)mc) {
+            oi = pay[P + t];
+            ov = pay[P + mc + t];
+        }
+        if (t == 0) fetch_head();
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const uint32_t k = t + i * kCT;
+            if (k < P) {
+                if (raw)
+                    sw[phys(k, lg)] = pv[i];
+                else
+                    pl[k] = pv[i];
+            }
+        }
+        __syncthreads();
+        if (!raw) {
+            // ranks of the bitmap words (G <= 128: warp 0, four words per lane)
             if (w == 0) {
                 uint32_t s4[4], tot = 0;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const uint32_t j = 4 * ln + i;
-                    s4[i] = (j < G) ? __popc(pay[j]) : 0u;
+                    s4[i] = (j < G) ? __popc(pl[j]) : 0u;
                     tot += s4[i];
                 }
                 uint32_t incl = tot;
@@ -339,64 +436,90 @@ __global__ void __launch_bounds__(kCT) chunk_decode(const ChunkedDecArgs a) {
                 uint32_t r0 = incl - tot;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    if (4 * ln + i < G) sm.rank[4 * ln + i] = r0;
+                    if (4 * ln + i < G) rank[4 * ln + i] = r0;
                     r0 += s4[i];
                 }
                 if (ln == 31 && G + incl != P) atomicOr(a.err, kErrCorrupt);  // the bitmap must account for P
             }
             __syncthreads();
             for (uint32_t k = t; k < mp; k += kCT) {
-                const uint32_t bw = pay[k / 32], bit = 1u << (k & 31u);
+                const uint32_t bw = pl[k / 32], bit = 1u << (k & 31u);
                 uint32_t v = 0;
                 if (bw & bit) {
-                    const uint32_t idx = G + sm.rank[k / 32] + __popc(bw & (bit - 1u));
-                    v = (idx < P) ? pay[idx] : 0u;
+                    const uint32_t idx = G + rank[k / 32] + __popc(bw & (bit - 1u));
+                    v = (idx < P) ? pl[idx] : 0u;
                 }
-                sm.sw[k] = v;
+                sw[phys(k, lg)] = v;
             }
+            __syncthreads();
         }
-        __syncthreads();
-        // inverse Bitshuffle: lane b holds plane b's word of group g; ballot l gives code l
-        for (uint32_t g = w; g < G; g += kCW) {
-            const uint32_t pw = sm.sw[ln * G + g];
-            uint32_t code = 0;
+        // inverse Bitshuffle (lane b: plane b's word -> lane l: code l), zigzag
+        // undone, inverse Diff: prefix sum over the chunk modulo 2^32
+        uint32_t vv[PER], run = 0;
 #pragma unroll
-            for (int l = 0; l < 32; ++l) {
-                const uint32_t cb = __ballot_sync(kFull, (pw >> l) & 1u);
-                if (ln == l) code = cb;
+        for (int i = 0; i < PER; ++i) {
+            const uint32_t g = first / 32 + i;
+            vv[i] = 0;
+            if (g >= G) continue;  // warp-uniform
+            uint32_t incl = (uint32_t)unzz(transpose32(sw[phys(ln * G + g, lg)], ln));
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t x = __shfl_up_sync(kFull, incl, o);
+                if (ln >= o) incl += x;
             }
-            sm.q[g * 32 + ln] = (uint32_t)unzz(code);
+            vv[i] = run + incl;
+            run += __shfl_sync(kFull, incl, 31);
         }
-        __syncthreads();
-        // inverse Diff: inclusive prefix sum over the chunk (modulo 2^32), then
-        // dequantization; thread t takes codes [t * E, t * E + E)
-        const uint32_t E = mp / kCT ? (mp + kCT - 1) / kCT : 1;
-        const uint32_t j0 = min(t * E, mp), j1 = min(j0 + E, mp);
-        uint32_t s = 0;
-        for (uint32_t j = j0; j < j1; ++j) s += sm.q[j];
-        uint32_t tot;
-        uint32_t run = block_excl(s, sm.tmp, &tot);
+        uint32_t all;
+        const uint32_t before = __shfl_sync(kFull, block_excl(ln == 0 ? run : 0u, tmp, &all), 0);
         float *gout = a.out + e0;
-        for (uint32_t j = j0; j < j1; ++j) {
-            run += sm.q[j];
-            if (j < cnt) gout[j] = __fmul_rn(__int2float_rn((int32_t)run), a.step);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const uint32_t j = first + 32 * i + ln;
+            if (j < cnt) gout[j] = __fmul_rn(__int2float_rn((int32_t)(vv[i] + before)), a.step);
         }
         __syncthreads();  // every reconstruction store of the chunk before its outliers
-        const uint32_t *oi = pay + P;
-        for (uint32_t k = t; k < mc; k += kCT) {
-            const uint32_t idx = oi[k], val = oi[mc + k];
+        if (t < (int)mc) {
+            if (oi >= e0 && oi < e0 + cnt)
+                a.out[oi] = __uint_as_float(ov);
+            else
+                atomicOr(a.err, kErrCorrupt);
+        }
+        for (uint32_t k = kCT + t; k < mc; k += kCT) {
+            const uint32_t idx = pay[P + k], val = pay[P + mc + k];
             if (idx >= e0 && idx < e0 + cnt)
                 a.out[idx] = __uint_as_float(val);
             else
                 atomicOr(a.err, kErrCorrupt);
         }
-        __syncthreads();
     }
 }
 
-int grid_for(uint64_t nc, int num_sms, int per_sm) {
+template <typename K>
+int grid_for(K kernel, size_t smem, uint64_t nc, int num_sms) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kCT, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
     const uint64_t want = (uint64_t)num_sms * per_sm;
     return (int)(nc < want ? (nc ? nc : 1) : want);
+}
+
+template <int PER>
+cudaError_t chunked_encode_as(const ChunkedArgs &a, int num_sms, cudaStream_t stream) {
+    const size_t es = enc_smem_bytes(a.m);
+    cudaError_t e = cudaFuncSetAttribute(chunk_encode<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)es);
+    if (e != cudaSuccess) return e;
+    if (a.nc) chunk_encode<PER><<<grid_for(chunk_encode<PER>, es, a.nc, num_sms), kCT, es, stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <int PER>
+cudaError_t chunked_decode_as(const ChunkedDecArgs &a, uint64_t nc, int num_sms, cudaStream_t stream) {
+    const size_t ds = dec_smem_bytes(a.m);
+    cudaError_t e = cudaFuncSetAttribute(chunk_decode<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ds);
+    if (e != cudaSuccess) return e;
+    if (nc) chunk_decode<PER><<<grid_for(chunk_decode<PER>, ds, nc, num_sms), kCT, ds, stream>>>(a);
+    return cudaGetLastError();
 }
 
 }  // namespace
@@ -404,24 +527,34 @@ int grid_for(uint64_t nc, int num_sms, int per_sm) {
 uint64_t chunked_slot_words(uint32_t m) { return 1 + (uint64_t)((m + 31) & ~31u) + 2ull * m; }
 
 cudaError_t launch_chunked_encode(const ChunkedArgs &a, int num_sms, cudaStream_t stream) {
-    const size_t es = sizeof(EncShared);
-    cudaError_t e = cudaFuncSetAttribute(chunk_encode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)es);
+    cudaError_t e;
+    switch (a.m) {
+    case 1024: e = chunked_encode_as<4>(a, num_sms, stream); break;
+    case 2048: e = chunked_encode_as<8>(a, num_sms, stream); break;
+    case 4096: e = chunked_encode_as<16>(a, num_sms, stream); break;
+    default: return cudaErrorInvalidValue;
+    }
     if (e != cudaSuccess) return e;
-    if (a.nc) chunk_encode<<<grid_for(a.nc, num_sms, 4), kCT, es, stream>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     chunk_scan<<<1, kScanThreads, 0, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (a.nc) chunk_gather<<<grid_for(a.nc, num_sms, 8), kCT, 0, stream>>>(a);
+    if (a.nc) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_gather, kCT, 0) != cudaSuccess || per_sm < 1)
+            per_sm = 1;
+        const uint64_t want = (uint64_t)num_sms * per_sm;
+        chunk_gather<<<(int)(a.nc < want ? a.nc : want), kCT, 0, stream>>>(a);
+    }
     return cudaGetLastError();
 }
 
 cudaError_t launch_chunked_decode(const ChunkedDecArgs &a, int num_sms, cudaStream_t stream) {
-    const size_t ds = sizeof(DecShared);
-    cudaError_t e = cudaFuncSetAttribute(chunk_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ds);
-    if (e != cudaSuccess) return e;
     const uint64_t nc = (a.n + a.m - 1) / a.m;
-    if (nc) chunk_decode<<<grid_for(nc, num_sms, 4), kCT, ds, stream>>>(a);
-    return cudaGetLastError();
+    switch (a.m) {
+    case 1024: return chunked_decode_as<4>(a, nc, num_sms, stream);
+    case 2048: return chunked_decode_as<8>(a, nc, num_sms, stream);
+    case 4096: return chunked_decode_as<16>(a, nc, num_sms, stream);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace eblc
