@@ -165,9 +165,33 @@ def workload(name: str, elements: int | None = None, rel=None, abs_=None, block=
 
 def workload_config(args, n, block, mode, bound, world):
     """The `config` both arms report for the same workload."""
-    return {"workload": args.workload if not args.elements else f"{args.workload}[:{n}]",
-            "n": int(n), "block": block, mode: bound, "parallelism": f"replicas{world}",
-            "l2": "flushed (256 MiB write, untimed) before every GPU compress and decompress call"}
+    c = {"workload": args.workload if not args.elements else f"{args.workload}[:{n}]", "n": int(n)}
+    if args.codec == "chunked":
+        c.update(codec="chunked", chunk_bytes=args.chunk)
+    else:
+        c["block"] = block
+        if args.lorenzo == "nd":
+            c.update(lorenzo="nd", dims=list(nd_dims(args)))
+    c.update({mode: bound, "parallelism": f"replicas{world}",
+              "l2": "flushed (256 MiB write, untimed) before every GPU compress and decompress call"})
+    return c
+
+
+def nd_dims(args):
+    """The workload's own 2-D / 3-D shape for lorenzo=nd (whole arrays only)."""
+    from error_bounded_lossy_encode_b200 import workloads as WL
+
+    d = WL.dims_of(args.workload)
+    if len(d) < 2 or args.elements:
+        raise SystemExit("--lorenzo nd needs a whole 2-D or 3-D workload")
+    return d
+
+
+def variant_suffix(args) -> str:
+    """'' for the default codec, else the codec's tag in profile file names."""
+    if args.codec == "chunked":
+        return f"_chunked{args.chunk}"
+    return "_nd" if args.lorenzo == "nd" else ""
 
 
 def host_info():
@@ -188,8 +212,12 @@ def host_info():
     return {"cpu_model": model, "cores_available": cores}
 
 
-def options_string(block, mode, bound, timing=False):
-    return f"{mode}={bound!r},block={block}" + (",timing=1" if timing else "")
+def options_string(block, mode, bound, timing=False, codec="block", chunk=16384, lorenzo="1d"):
+    if codec == "chunked":
+        o = f"{mode}={bound!r},codec=chunked,chunk={chunk}"
+    else:
+        o = f"{mode}={bound!r},block={block}" + (",lorenzo=nd" if lorenzo == "nd" else "")
+    return o + (",timing=1" if timing else "")
 
 
 def measured_peak():
@@ -227,20 +255,36 @@ def profiled_traffic(kernel: str, workload_name: str):
 # ----------------------------------------------------------------------------------------------
 # CPU oracle legs
 
-def cpu_oracle_sample(x, block, mode, bound, repeats=1, all_cores=False, elems=CPU_SAMPLE_ELEMS):
+def cpu_oracle_sample(x, block, mode, bound, repeats=1, all_cores=False, elems=CPU_SAMPLE_ELEMS, codec="block",
+                      chunk=16384, dims=None):
     """Time the CPU oracle (compress + decompress) on the first `elems`
     elements: the plain single-threaded oracle, or (all_cores) the OpenMP
-    build of the same steps."""
+    build of the same steps (block codec, 1-D Lorenzo).  With dims (lorenzo
+    nd) the sample is whole leading slabs of the array."""
     import oracle
 
     oracle.build()
-    comp, decomp = (oracle.compress_omp, oracle.decompress_omp) if all_cores else \
-        (oracle.compress, oracle.decompress)
+    if all_cores and (codec != "block" or dims):
+        return None
     s = x[:elems]
+    if codec == "chunked":
+        comp = lambda v, **b: oracle.compress_chunked(v, chunk, **b)
+        decomp = oracle.decompress
+    elif dims:
+        slab = int(np.prod(dims[1:]))
+        edge = 16 if len(dims) == 3 else 64  # whole bricks along the slowest axis
+        k = max(edge, min(dims[0], elems // slab) // edge * edge)
+        s = x[:k * slab]
+        comp = lambda v, **b: oracle.compress_lorenzo(v.reshape((k,) + tuple(dims[1:])), block, **b)
+        decomp = oracle.decompress
+    else:
+        comp0, decomp = (oracle.compress_omp, oracle.decompress_omp) if all_cores else \
+            (oracle.compress, oracle.decompress)
+        comp = lambda v, **b: comp0(v, block, **b)
     t_c = t_d = 0.0
     for _ in range(repeats):
         t0 = time.perf_counter()
-        stream = comp(s, block, **{mode: bound})
+        stream = comp(s, **{mode: bound})
         t1 = time.perf_counter()
         decomp(stream, s.size)
         t2 = time.perf_counter()
@@ -249,16 +293,23 @@ def cpu_oracle_sample(x, block, mode, bound, repeats=1, all_cores=False, elems=C
     gbs = repeats * 4 * s.size / (t_c + t_d) / 1e9
     cores = oracle.omp_threads() if all_cores else 1
     what = f"the oracle's steps run over chunks with OpenMP on {cores} threads" if all_cores else \
-        "single-threaded plain C oracle"
+        "single-threaded plain C oracle" + (f", chunked codec ({chunk}-byte chunks)" if codec == "chunked" else
+                                            ", multi-dimensional Lorenzo" if dims else "")
     part = "the whole workload" if s.size == x.size else f"first {s.size} elements ({4 * s.size >> 20} MiB) of the workload"
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
             "kind": "oracle" if not all_cores else "oracle (all-core OpenMP build)",
             "sample": f"{part}, compress+decompress, {what}",
+            "elements": int(s.size),
             "compress_gbs": round(repeats * 4 * s.size / t_c / 1e9, 4),
             "decompress_gbs": round(repeats * 4 * s.size / t_d / 1e9, 4)}
 
 
 REFERENCE_BUDGET_S = 150.0  # wall-time budget of the reference arm's timed steps
+
+
+def oracle_kwargs(args) -> dict:
+    return {"codec": args.codec, "chunk": args.chunk,
+            "dims": nd_dims(args) if args.codec == "block" and args.lorenzo == "nd" else None}
 
 
 def run_reference(args):
@@ -270,19 +321,23 @@ def run_reference(args):
     if rank != 0:
         return 0
     x, block, mode, bound = workload(args.workload, args.elements, args.rel, args.abs, args.block)
-    probe = cpu_oracle_sample(x, block, mode, bound, elems=1 << 22)
+    kw = oracle_kwargs(args)
+    probe = cpu_oracle_sample(x, block, mode, bound, elems=1 << 22, **kw)
     est_step_s = 4.0 * x.size / (probe["value"] * 1e9)
     elems = x.size if est_step_s * args.steps <= REFERENCE_BUDGET_S else \
         max(1 << 22, int(REFERENCE_BUDGET_S / args.steps * probe["value"] * 1e9 / 4) // 4096 * 4096)
     warm = args.warmup if est_step_s * (args.steps + args.warmup) <= 1.5 * REFERENCE_BUDGET_S else 1
     for _ in range(warm):
-        cpu_oracle_sample(x, block, mode, bound, elems=min(elems, 1 << 22))
+        cpu_oracle_sample(x, block, mode, bound, elems=min(elems, 1 << 22), **kw)
     t0 = time.perf_counter()
-    base = cpu_oracle_sample(x, block, mode, bound, repeats=args.steps, elems=elems)
+    base = cpu_oracle_sample(x, block, mode, bound, repeats=args.steps, elems=elems, **kw)
     elapsed = time.perf_counter() - t0
     config = workload_config(args, x.size, block, mode, bound, world)
-    if elems < x.size:
-        config = dict(config, workload=f"{config['workload']}[:{elems}]", n=int(elems))
+    if base["elements"] < x.size:
+        config = dict(config, workload=f"{config['workload']}[:{base['elements']}]", n=int(base["elements"]))
+        if kw["dims"]:  # whole leading slabs of the array
+            d = list(kw["dims"])
+            config["dims"] = [base["elements"] // int(np.prod(d[1:]))] + d[1:]
     line = {"metric": METRIC, "value": base["value"], "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(1e3 * elapsed / max(1, args.steps), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
@@ -317,7 +372,10 @@ def run_ours(args):
 
     x_np, block, mode, bound = workload(args.workload, args.elements, args.rel, args.abs, args.block)
     n = x_np.size
-    st, plan = E.eblc_plan_create([n], None, options_string(block, mode, bound, timing=True))
+    kw = oracle_kwargs(args)
+    dims = list(kw["dims"]) if kw["dims"] else [n]
+    st, plan = E.eblc_plan_create(dims, None, options_string(block, mode, bound, True, args.codec, args.chunk,
+                                                              args.lorenzo))
     if st != E.EBLC_OK:
         raise RuntimeError("plan_create: " + E.STATUS_NAMES[st])
     _, lim = E.eblc_plan_get_limits(plan)
@@ -330,7 +388,8 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
     ex = E.cuda_exec(stream.cuda_stream)
     sc = E.eblc_sidecar_t()
-    launches_per_step = (3 if mode == "rel" else 2) + 1  # [range,] encode, finish; decode
+    # [range,] encode (chunked: encode, scan, gather), finish; decode
+    launches_per_step = (1 if mode == "rel" else 0) + (3 if args.codec == "chunked" else 1) + 1 + 1
 
     def step(timed):
         flush.fill_(1)
@@ -393,7 +452,8 @@ def run_ours(args):
                                  med(dec_dev)], world, dev)))
     step_bytes = sum_over_ranks([4.0 * n], world, dev)[0]
 
-    graph = run_graph_compress(E, plan, x, out, cap, flush, nbytes, args, world, dev)
+    graph = run_graph_compress(E, plan, x, out, cap, flush, nbytes, args, world, dev) if args.codec == "block" \
+        else {"error": "the chunked codec has its synchronous calls only"}
 
     # e2e: HOST execution kind, pinned host buffers, copies inside the timed region
     e2e = None
@@ -584,8 +644,10 @@ def report(args, world, n, nbytes, T, step_bytes, kern, e2e, launches_per_step, 
         kstats[k] = {"avg_ms": round(avg_ms, 4), "median_ms": round(float(np.median(v)), 4), "launches": len(v),
                      "algorithmic_bytes": int(algo[k]), "achieved_gbs": round(ach, 1),
                      "frac_of_measured_peak": round(ach / peak, 4)}
+    if args.codec == "chunked":
+        kstats["encode"]["what"] = "chunk_encode + chunk_scan + chunk_gather (one timing mark around the three)"
     dom = max(kstats, key=lambda k: kstats[k]["avg_ms"])
-    traffic = profiled_traffic(dom, args.workload)
+    traffic = profiled_traffic(dom, args.workload + variant_suffix(args))
     line = {
         "metric": METRIC,
         "value": round(step_bytes / T["step"] / 1e9, 2),
@@ -628,8 +690,11 @@ def report(args, world, n, nbytes, T, step_bytes, kern, e2e, launches_per_step, 
                         "bound by launch and host synchronisation latency, not HBM (graph_compress shows the "
                         "sync-free form)")
     if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_oracle_sample(x_np, block, mode, bound)
-        line["cpu_baseline_all_cores"] = cpu_oracle_sample(x_np, block, mode, bound, all_cores=True)
+        kw = oracle_kwargs(args)
+        line["cpu_baseline"] = cpu_oracle_sample(x_np, block, mode, bound, **kw)
+        allc = cpu_oracle_sample(x_np, block, mode, bound, all_cores=True, **kw)
+        line["cpu_baseline_all_cores"] = allc if allc is not None else \
+            {"unavailable": "the OpenMP oracle build covers the block codec with the 1-D predictor only"}
         line["host"] = host_info()
     print(json.dumps(line), flush=True)
 
@@ -647,9 +712,19 @@ def main(argv=None):
     ap.add_argument("--rel", type=float, default=None, help="override the workload's bound: relative")
     ap.add_argument("--abs", type=float, default=None, help="override the workload's bound: absolute")
     ap.add_argument("--block", type=int, default=None, choices=(32, 64, 128, 256), help="override the block size")
+    ap.add_argument("--codec", choices=("block", "chunked"), default="block",
+                    help="block: the fused block codec (default); chunked: the chunk-cooperative codec")
+    ap.add_argument("--chunk", type=int, choices=(4096, 8192, 16384), default=16384,
+                    help="bytes of input per chunk of the chunked codec")
+    ap.add_argument("--lorenzo", choices=("1d", "nd"), default="1d",
+                    help="nd: the 2-D / 3-D Lorenzo predictor over the workload's own shape")
     ap.add_argument("--sharded", action="store_true",
                     help="split one array across the ranks (range all-reduce; strong scaling) instead of replicas")
     args = ap.parse_args(argv)
+    if args.codec == "chunked" and args.lorenzo == "nd":
+        ap.error("--lorenzo nd belongs to the block codec")
+    if args.sharded and (args.codec != "block" or args.lorenzo != "1d"):
+        ap.error("--sharded runs the block codec with the 1-D predictor")
     if args.impl == "reference":
         return run_reference(args)
     if args.sharded:

@@ -157,6 +157,12 @@ def options_of(name: str) -> dict:
     return dict(STANDARD[name][2])
 
 
+def dims_of(name: str) -> tuple[int, ...]:
+    """The workload's array shape, slowest axis first ((n,) for 1-D ones)."""
+    kw = STANDARD[name][1]
+    return tuple(kw["shape"]) if "shape" in kw else (int(kw["n"]),)
+
+
 def sha256(x: np.ndarray) -> str:
     return hashlib.sha256(np.ascontiguousarray(x).view(np.uint8)).hexdigest()
 

@@ -68,6 +68,9 @@ class _Args:
     rel = None
     abs = None
     block = None
+    codec = "block"
+    chunk = 16384
+    lorenzo = "1d"
 
 
 def test_report_line_contract(monkeypatch):
@@ -124,3 +127,22 @@ def test_host_info_names_cpu_and_cores():
     h = bench.host_info()
     assert h["cores_available"] >= 1
     assert "cpu_model" in h
+
+
+def test_codec_variants_name_themselves():
+    """--codec chunked and --lorenzo nd: the plan options and the config say
+    which codec or predictor was timed (both arms build the config alike)."""
+    class Ch(_Args):
+        codec, chunk = "chunked", 4096
+
+    class Nd(_Args):
+        lorenzo = "nd"
+
+    c = bench.workload_config(Ch, 1 << 20, 64, "rel", 1e-3, 1)
+    assert c["codec"] == "chunked" and c["chunk_bytes"] == 4096 and "block" not in c
+    assert bench.options_string(64, "rel", 1e-3, False, "chunked", 4096) == "rel=0.001,codec=chunked,chunk=4096"
+    d = bench.workload_config(Nd, 1 << 27, 64, "rel", 1e-3, 1)
+    assert d["lorenzo"] == "nd" and d["dims"] == [512, 512, 512] and d["block"] == 64
+    assert bench.options_string(64, "rel", 1e-3, False, "block", 16384, "nd") == "rel=0.001,block=64,lorenzo=nd"
+    assert bench.variant_suffix(Ch) == "_chunked4096" and bench.variant_suffix(Nd) == "_nd"
+    assert bench.variant_suffix(_Args) == ""
