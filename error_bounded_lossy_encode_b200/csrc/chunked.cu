@@ -5,23 +5,28 @@
 // File Reference", launchNvrtcChunkFusedEncode: each chunk's coded form in a
 // scratch slot with its size, then the cross-chunk scan/pack tail).
 //
-//   chunk_encode  one CTA per chunk (grid-stride), each warp a contiguous run
-//                 of 32-code groups in registers: the linear quantizer and
-//                 the outlier test, first differences reset at the chunk start
-//                 in zigzag form, the 32 x 32 bit transpose of every group
-//                 (lane b gets bit plane b) by a shuffle butterfly, zero
-//                 elimination (a bitmap of the nonzero words by ballots, the
-//                 nonzero words compacted warp by warp after one block scan)
-//                 or the shuffled words verbatim when that is not smaller,
-//                 then the chunk's outliers in ascending order; the record
-//                 goes to the chunk's scratch slot, its size to sizes[].
-//   chunk_scan    one CTA: exclusive scan of the record sizes and outlier
-//                 counts -> chunk index, header and result block.
-//   chunk_gather  records from scratch to their place in the stream.
-//   chunk_decode  one CTA per chunk: zero elimination undone (ranks by
-//                 popcounts), the inverse transpose, zigzag undone and the
-//                 prefix sum in each warp's registers, one block scan of the
-//                 warps' totals, dequantization, outliers.
+//   chunk_encode  one CTA per chunk, each CTA a contiguous range of chunks,
+//                 each warp a contiguous run of 32-code groups in registers:
+//                 the linear quantizer and the outlier test, first
+//                 differences reset at the chunk start in zigzag form, the
+//                 32 x 32 bit transpose of every group (lane b gets bit plane
+//                 b) by a shuffle butterfly, zero elimination (a bitmap of the
+//                 nonzero words by ballots, the nonzero words compacted warp
+//                 by warp after one block scan) or the shuffled words
+//                 verbatim when that is not smaller, then the chunk's
+//                 outliers in ascending order; the record goes to the chunk's
+//                 scratch slot, its size to sizes[], the range's totals to
+//                 part[].
+//   chunk_scan    one CTA: exclusive scan of the chunk ranges' record words
+//                 and outlier counts -> range bases, header, result block.
+//   chunk_gather  one CTA per chunk range: the chunk index entries (a block
+//                 scan from the range's base), records from scratch to their
+//                 place in the stream.
+//   chunk_decode  one CTA per chunk: zero elimination undone (each warp a
+//                 run of bitmap words, ranks by popcounts), the inverse
+//                 transpose, zigzag undone and the prefix sum in each warp's
+//                 registers, one block scan of the warps' totals,
+//                 dequantization, outliers.
 // No inter-CTA waits anywhere: the scan is its own launch.
 #include "common.cuh"
 #include "kernels.h"
@@ -50,6 +55,24 @@ __device__ __forceinline__ uint32_t transpose32(uint32_t w, int ln) {
     }
     return w;
 }
+// The same transpose when the codes use bit planes 0..3 only (codes < 16):
+// four ballots, lane b < 4 keeps plane b, the other lanes' planes are 0.
+__device__ __forceinline__ uint32_t transpose32_low4(uint32_t d, int ln) {
+    const uint32_t p0 = __ballot_sync(kFull, d & 1u), p1 = __ballot_sync(kFull, d & 2u);
+    const uint32_t p2 = __ballot_sync(kFull, d & 4u), p3 = __ballot_sync(kFull, d & 8u);
+    const uint32_t lo = (ln & 1) ? p1 : p0, hi = (ln & 1) ? p3 : p2;
+    return (ln >= 4) ? 0u : ((ln & 2) ? hi : lo);
+}
+
+// Inverse transpose when only planes 0..nb-1 (lanes 0..nb-1) may be nonzero:
+// lane l collects bit l of each plane word.
+__device__ __forceinline__ uint32_t untranspose32_low(uint32_t pw, int nb, int ln) {
+    uint32_t code = 0;
+#pragma unroll 4
+    for (int b = 0; b < nb; ++b) code |= ((__shfl_sync(kFull, pw, b) >> ln) & 1u) << b;
+    return code;
+}
+
 __device__ __forceinline__ int32_t unzz(uint32_t z) { return (int32_t)((z >> 1) ^ (0u - (z & 1u))); }
 
 // Exclusive block-wide prefix of v (every thread of the CTA calls it);
@@ -99,16 +122,24 @@ __device__ __forceinline__ int32_t quant(const Bound &bd, float x, bool &o) {
     return qq;
 }
 
+// Quantized code alone (the quantizer's range rule included).
+__device__ __forceinline__ int32_t quant_code(const Bound &bd, float x) {
+    const float y = __fmul_rn(x, bd.inv2eb);
+    return (fabsf(y) < 0x1p30f) ? __float2int_rn(y) : 0;
+}
+
 // Dynamic shared memory of the encoder for chunks of m elements: the
 // shuffled words, the outlier flag words, the scan's warp totals.
 __host__ __device__ constexpr size_t enc_smem_bytes(uint32_t m) { return 4ull * (m + m / 32 + kCW); }
 
-// PER = m / kCT.  Warp w owns the PER groups of 32 codes starting at code
-// 32 PER w of the chunk and keeps them in registers from the load to the
-// bit transpose; the input of the CTA's next chunk is loaded as soon as the
-// current chunk's codes are formed, so its latency overlaps the rest.
+// PER = m / kCT.  CTA b codes the chunks [b K, b K + K) (K = per_range) in
+// order and leaves their total record words and outliers in part[].  Warp w
+// owns the PER groups of 32 codes starting at code 32 PER w of the chunk and
+// keeps them in registers from the load to the bit transpose; the input of
+// the CTA's next chunk is loaded as soon as the current chunk's codes are
+// formed, so its latency overlaps the rest.
 template <int PER>
-__global__ void __launch_bounds__(kCT) chunk_encode(const ChunkedArgs a) {
+__global__ void __launch_bounds__(kCT, PER == 4 ? 6 : PER == 8 ? 4 : 3) chunk_encode(const ChunkedArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint32_t *const sw = reinterpret_cast<uint32_t *>(smem_raw);
     uint32_t *const oflag = sw + a.m;
@@ -133,9 +164,11 @@ __global__ void __launch_bounds__(kCT) chunk_encode(const ChunkedArgs a) {
         // the code before the warp's first one (its difference), re-quantized here
         xp = (ln == 0 && first > 0 && first <= cnt) ? a.in[e0 + first - 1] : 0.0f;
     };
-    load(blockIdx.x);
+    const uint64_t cb = (uint64_t)blockIdx.x * a.per_range, ce = min(a.nc, cb + a.per_range);
+    uint32_t tot_r = 0, tot_m = 0;  // thread 0: the range's record words and outliers
+    load(cb);
     __syncthreads();
-    for (uint64_t c = blockIdx.x; c < a.nc; c += gridDim.x) {
+    for (uint64_t c = cb; c < ce; ++c) {
         const uint64_t e0 = c * a.m;
         const uint32_t cnt = (uint32_t)min((uint64_t)a.m, a.n - e0), mp = (cnt + 31u) & ~31u, G = mp / 32;
         const int lg = (mp == a.m) ? lg_full : 0;
@@ -143,24 +176,34 @@ __global__ void __launch_bounds__(kCT) chunk_encode(const ChunkedArgs a) {
         // Quant, Diff (zigzag, reset at the chunk start) and Bitshuffle of the
         // warp's groups: lane l holds code 32 g + l; the transpose gives lane b
         // plane b's word of the group.
-        bool o;
+        // The fp32 filter settles almost every code; a warp with any element
+        // not certainly within the bound (or possibly out of range) redoes
+        // its group with the quantizer's range rule and the exact test.
+        const uint32_t sx = (mp == a.m) ? (uint32_t)ln : 0u;  // phys(ln G + g) for this lane
+        const bool chk = bd.check_range != 0;
         int32_t prev = 0;
-        if (ln == 0 && first > 0 && first <= cnt) prev = quant(bd, xp, o);
+        if (ln == 0 && first > 0 && first <= cnt) prev = quant_code(bd, xp);
 #pragma unroll
         for (int i = 0; i < PER; ++i) {
             const uint32_t g = first / 32 + i, j = 32 * g + ln;
             if (g >= G) break;  // warp-uniform
-            o = false;
-            const int32_t qq = (j < cnt) ? quant(bd, xv[i], o) : 0;
+            const float x = xv[i];  // 0 past the chunk's end
+            const float y = __fmul_rn(x, bd.inv2eb);
+            int32_t qq = __float2int_rn(y);
+            const float xr = __fmul_rn(__int2float_rn(qq), bd.step);
+            const bool flag = !(fabsf(__fsub_rn(x, xr)) <= bd.t_in) || (chk && !(fabsf(y) < 0x1p30f));
+            bool o = false;
+            if (__any_sync(kFull, flag)) qq = (j < cnt) ? quant(bd, x, o) : 0;
             int32_t left = __shfl_up_sync(kFull, qq, 1);
             if (ln == 0) left = prev;
             prev = __shfl_sync(kFull, qq, 31);
             const uint32_t d = (j < cnt) ? zz(qq - left) : 0u;
             const uint32_t fw = __ballot_sync(kFull, o);
             if (ln == 0) oflag[g] = fw;
-            sw[phys(ln * G + g, lg)] = transpose32(d, ln);
+            const uint32_t wide = __reduce_or_sync(kFull, d) >> 4;  // any code using plane 4 or above
+            sw[ln * G + (g ^ sx)] = wide ? transpose32(d, ln) : transpose32_low4(d, ln);
         }
-        load(c + gridDim.x);
+        load(c + 1 < ce ? c + 1 : a.nc);
         __syncthreads();
         // One block scan for both counts: warp w's nonzero words over its word
         // range [k0, k1) (upper 16 bits, lane 0 only) and thread t's outliers
@@ -204,37 +247,44 @@ __global__ void __launch_bounds__(kCT) chunk_encode(const ChunkedArgs a) {
             rec[0] = P | (raw ? 0x80000000u : 0u);
             a.sizes[c] = 1 + P + 2 * mc;
             a.outl[c] = mc;
+            tot_r += 1 + P + 2 * mc;
+            tot_m += mc;
         }
         __syncthreads();
+    }
+    if (t == 0) {
+        a.part[blockIdx.x] = tot_r;
+        a.part[a.nc + blockIdx.x] = tot_m;
     }
 }
 
 constexpr int kScanThreads = 1024;
 constexpr int kScanWarps = kScanThreads / 32;
 
-// Exclusive scan of the record sizes and outlier counts over all chunks (one
-// CTA), the chunk index and the header of the stream, the result block.
-// Warp w takes a contiguous range of chunks, 32 at a time (coalesced): one
-// pass for the warps' totals, a scan of those, a second pass for the entries.
+// Exclusive scan of the chunk ranges' totals (one CTA; part[] is replaced
+// by the ranges' bases), the header of the stream, the result block.
 __global__ void __launch_bounds__(kScanThreads) chunk_scan(const ChunkedArgs a) {
     __shared__ unsigned long long part_r[kScanWarps], part_m[kScanWarps];
     const int t = threadIdx.x, ln = t % 32, w = t / 32;
-    const uint64_t steps = (a.nc + 32 * kScanWarps - 1) / (32 * kScanWarps);  // 32-chunk steps per warp
-    const uint64_t c0 = min(a.nc, (uint64_t)w * steps * 32), c1 = min(a.nc, c0 + steps * 32);
+    const uint32_t per = (a.ranges + kScanThreads - 1) / kScanThreads;  // ranges per thread
+    const uint32_t b0 = min(a.ranges, per * t), b1 = min(a.ranges, b0 + per);
     unsigned long long sr = 0, sm_ = 0;
-#pragma unroll 4
-    for (uint64_t c = c0 + ln; c < c1; c += 32) {
-        sr += a.sizes[c];
-        sm_ += a.outl[c];
+    for (uint32_t b = b0; b < b1; ++b) {
+        sr += a.part[b];
+        sm_ += a.part[a.nc + b];
     }
+    unsigned long long ir = sr, im = sm_;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
-        sr += __shfl_xor_sync(kFull, sr, o);
-        sm_ += __shfl_xor_sync(kFull, sm_, o);
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long x = __shfl_up_sync(kFull, ir, o), y = __shfl_up_sync(kFull, im, o);
+        if (ln >= o) {
+            ir += x;
+            im += y;
+        }
     }
-    if (ln == 0) {
-        part_r[w] = sr;
-        part_m[w] = sm_;
+    if (ln == 31) {
+        part_r[w] = ir;
+        part_m[w] = im;
     }
     __syncthreads();
     unsigned long long r = 0, m = 0, R = 0, M = 0;
@@ -244,28 +294,17 @@ __global__ void __launch_bounds__(kScanThreads) chunk_scan(const ChunkedArgs a) 
         R += part_r[k];
         M += part_m[k];
     }
+    r += ir - sr;
+    m += im - sm_;
+    for (uint32_t b = b0; b < b1; ++b) {
+        const uint32_t xr = a.part[b], xm = a.part[a.nc + b];
+        a.part[b] = (uint32_t)r;
+        a.part[a.nc + b] = (uint32_t)m;
+        r += xr;
+        m += xm;
+    }
     const Layout L = chunked_layout(a.n, a.m);
     const bool idx_fits = L.record_off <= a.out_cap;
-    for (uint64_t cb = c0; cb < c1; cb += 32) {
-        const uint64_t c = cb + ln;
-        const uint32_t s = (c < c1) ? a.sizes[c] : 0u, q = (c < c1) ? a.outl[c] : 0u;
-        uint32_t is = s, iq = q;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t x = __shfl_up_sync(kFull, is, o), y = __shfl_up_sync(kFull, iq, o);
-            if (ln >= o) {
-                is += x;
-                iq += y;
-            }
-        }
-        const uint64_t rc = r + is - s, mcc = m + iq - q;
-        if (c < c1) {
-            a.offs[c] = (uint32_t)rc;
-            if (idx_fits) *reinterpret_cast<uint2 *>(a.out + L.index_off + 8 * c) = make_uint2((uint32_t)rc, (uint32_t)mcc);
-        }
-        r += __shfl_sync(kFull, is, 31);
-        m += __shfl_sync(kFull, iq, 31);
-    }
     if (t != 0) return;
     const float vmin = a.abs_mode ? 0.0f : a.range[0], vmax = a.abs_mode ? 0.0f : a.range[1];
     const Bound bd = resolve_bound(a.abs_mode, a.bound, vmin, vmax);
@@ -308,22 +347,46 @@ __global__ void __launch_bounds__(kScanThreads) chunk_scan(const ChunkedArgs a) 
     for (uint64_t b = L.index_off + 8 * a.nc; b < L.record_off; b += 4) *reinterpret_cast<uint32_t *>(a.out + b) = 0u;
 }
 
+// CTA b: the chunk index entries of range b (a block scan of its chunks'
+// sizes from the range's base, 256 chunks at a time), then the records from
+// their scratch slots to their offsets, one warp per chunk.
 __global__ void __launch_bounds__(kCT) chunk_gather(const ChunkedArgs a) {
+    __shared__ uint32_t off_s[kCT], len_s[kCT], tmp[kCW];
+    const int t = threadIdx.x, ln = t % 32, w = t / 32;
     const Layout L = chunked_layout(a.n, a.m);
     uint32_t *recs = reinterpret_cast<uint32_t *>(a.out + L.record_off);
     const uint64_t cap_words = (a.out_cap > L.record_off) ? (a.out_cap - L.record_off) / 4 : 0;
-    for (uint64_t c = blockIdx.x; c < a.nc; c += gridDim.x) {
-        const uint64_t o = a.offs[c], len = a.sizes[c];
-        if (o + len > cap_words) continue;  // reported by chunk_scan (capacity)
-        const uint32_t *src = a.scratch + c * (uint64_t)a.slot_words;
-        for (uint64_t k = threadIdx.x; k < len; k += kCT) st_cs_u32(recs + o + k, src[k]);
+    const bool idx_fits = L.record_off <= a.out_cap;
+    const uint64_t cb = (uint64_t)blockIdx.x * a.per_range, ce = min(a.nc, cb + a.per_range);
+    uint32_t base_r = a.part[blockIdx.x], base_m = a.part[a.nc + blockIdx.x];
+    for (uint64_t c0 = cb; c0 < ce; c0 += kCT) {
+        const uint64_t c = c0 + t;
+        const uint32_t s = (c < ce) ? a.sizes[c] : 0u, q = (c < ce) ? a.outl[c] : 0u;
+        uint32_t tr, tm;
+        const uint32_t er = block_excl(s, tmp, &tr);
+        const uint32_t em = block_excl(q, tmp, &tm);
+        if (c < ce && idx_fits)
+            *reinterpret_cast<uint2 *>(a.out + L.index_off + 8 * c) = make_uint2(base_r + er, base_m + em);
+        off_s[t] = base_r + er;
+        len_s[t] = s;
+        __syncthreads();
+        const uint32_t nw = (uint32_t)min((uint64_t)kCT, ce - c0);
+        for (uint32_t k = w; k < nw; k += kCW) {
+            const uint64_t o = off_s[k], len = len_s[k];
+            if (o + len > cap_words) continue;  // reported by chunk_scan (capacity)
+            const uint32_t *src = a.scratch + (c0 + k) * (uint64_t)a.slot_words;
+            for (uint32_t j = ln; j < len; j += 32) st_cs_u32(recs + o + j, src[j]);
+        }
+        base_r += tr;
+        base_m += tm;
+        __syncthreads();
     }
 }
 
 // Dynamic shared memory of the decoder for chunks of m elements: the record's
-// payload words, the shuffled words, the ranks of the bitmap words, the
-// scan's warp totals and the chunk's record facts.
-__host__ __device__ constexpr size_t dec_smem_bytes(uint32_t m) { return 4ull * (2 * m + m / 32 + kCW + 4); }
+// payload words, the shuffled words, the scan's warp totals and the chunk's
+// record facts.
+__host__ __device__ constexpr size_t dec_smem_bytes(uint32_t m) { return 4ull * (2 * m + kCW + 4); }
 
 // PER = m / kCT.  Warp w decodes the PER groups starting at code 32 PER w:
 // the transpose, zigzag and the prefix sum stay in its registers, and its
@@ -331,12 +394,11 @@ __host__ __device__ constexpr size_t dec_smem_bytes(uint32_t m) { return 4ull * 
 // entries and the head word of the CTA's next chunk one chunk ahead; the
 // payload and the first kCT outliers of a chunk come in one round of loads.
 template <int PER>
-__global__ void __launch_bounds__(kCT) chunk_decode(const ChunkedDecArgs a) {
+__global__ void __launch_bounds__(kCT, PER == 4 ? 5 : PER == 8 ? 4 : 3) chunk_decode(const ChunkedDecArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint32_t *const pl = reinterpret_cast<uint32_t *>(smem_raw);  // payload (RZE form)
     uint32_t *const sw = pl + a.m;
-    uint32_t *const rank = sw + a.m;
-    uint32_t *const tmp = rank + a.m / 32;
+    uint32_t *const tmp = sw + a.m;
     uint32_t *const info = tmp + kCW;  // P (0xffffffff: corrupt), raw, mc, record word offset
     const int t = threadIdx.x, ln = t % 32, w = t / 32;
     const int lg_full = 31 - __clz(a.m / 32);
@@ -373,6 +435,7 @@ __global__ void __launch_bounds__(kCT) chunk_decode(const ChunkedDecArgs a) {
         const uint64_t e0 = c * a.m;
         const uint32_t cnt = (uint32_t)min((uint64_t)a.m, a.n - e0), mp = (cnt + 31u) & ~31u, G = mp / 32;
         const int lg = (mp == a.m) ? lg_full : 0;
+        const uint32_t sx = (mp == a.m) ? (uint32_t)ln : 0u;
         if (t == 0) {
             uint32_t P = head & 0x7fffffffu, raw = head >> 31, mc = (uint32_t)(ny - ey);
             const bool ok = eok && ex + 1 + P + 2ull * mc == nx && (raw ? P == mp : (P >= G && P < mp));
@@ -418,39 +481,26 @@ __global__ void __launch_bounds__(kCT) chunk_decode(const ChunkedDecArgs a) {
         }
         __syncthreads();
         if (!raw) {
-            // ranks of the bitmap words (G <= 128: warp 0, four words per lane)
-            if (w == 0) {
-                uint32_t s4[4], tot = 0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t j = 4 * ln + i;
-                    s4[i] = (j < G) ? __popc(pl[j]) : 0u;
-                    tot += s4[i];
-                }
-                uint32_t incl = tot;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t x = __shfl_up_sync(kFull, incl, o);
-                    if (ln >= o) incl += x;
-                }
-                uint32_t r0 = incl - tot;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    if (4 * ln + i < G) rank[4 * ln + i] = r0;
-                    r0 += s4[i];
-                }
-                if (ln == 31 && G + incl != P) atomicOr(a.err, kErrCorrupt);  // the bitmap must account for P
-            }
-            __syncthreads();
-            for (uint32_t k = t; k < mp; k += kCT) {
-                const uint32_t bw = pl[k / 32], bit = 1u << (k & 31u);
+            // zero elimination undone: warp w expands the bitmap words [j0, j1)
+            // (in order), its first nonzero word's rank the popcount of the
+            // bitmap words before j0
+            const uint32_t per = (G + kCW - 1) / kCW;
+            const uint32_t j0 = min(w * per, G), j1 = min(j0 + per, G);
+            uint32_t base = 0;
+            for (uint32_t j = ln; j < j0; j += 32) base += __popc(pl[j]);
+            base = __reduce_add_sync(kFull, base);
+            const uint32_t lt = (1u << ln) - 1u;
+            for (uint32_t j = j0; j < j1; ++j) {
+                const uint32_t bw = pl[j];
                 uint32_t v = 0;
-                if (bw & bit) {
-                    const uint32_t idx = G + rank[k / 32] + __popc(bw & (bit - 1u));
+                if ((bw >> ln) & 1u) {
+                    const uint32_t idx = G + base + __popc(bw & lt);
                     v = (idx < P) ? pl[idx] : 0u;
                 }
-                sw[phys(k, lg)] = v;
+                sw[phys(32 * j + ln, lg)] = v;
+                base += __popc(bw);
             }
+            if (j1 == G && j0 < j1 && ln == 0 && G + base != P) atomicOr(a.err, kErrCorrupt);  // the bitmap must account for P
             __syncthreads();
         }
         // inverse Bitshuffle (lane b: plane b's word -> lane l: code l), zigzag
@@ -461,7 +511,9 @@ __global__ void __launch_bounds__(kCT) chunk_decode(const ChunkedDecArgs a) {
             const uint32_t g = first / 32 + i;
             vv[i] = 0;
             if (g >= G) continue;  // warp-uniform
-            uint32_t incl = (uint32_t)unzz(transpose32(sw[phys(ln * G + g, lg)], ln));
+            const uint32_t pw = sw[ln * G + (g ^ sx)];
+            const int nb = 32 - __clz(__ballot_sync(kFull, pw != 0u));  // planes 0..nb-1 may be nonzero
+            uint32_t incl = (uint32_t)unzz(nb > 12 ? transpose32(pw, ln) : untranspose32_low(pw, nb, ln));
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const uint32_t x = __shfl_up_sync(kFull, incl, o);
@@ -504,12 +556,20 @@ int grid_for(K kernel, size_t smem, uint64_t nc, int num_sms) {
     return (int)(nc < want ? (nc ? nc : 1) : want);
 }
 
+// One contiguous chunk range per CTA of one resident wave.
 template <int PER>
-cudaError_t chunked_encode_as(const ChunkedArgs &a, int num_sms, cudaStream_t stream) {
+cudaError_t chunked_encode_as(ChunkedArgs a, int num_sms, cudaStream_t stream) {
     const size_t es = enc_smem_bytes(a.m);
     cudaError_t e = cudaFuncSetAttribute(chunk_encode<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)es);
     if (e != cudaSuccess) return e;
-    if (a.nc) chunk_encode<PER><<<grid_for(chunk_encode<PER>, es, a.nc, num_sms), kCT, es, stream>>>(a);
+    const uint64_t want = (uint64_t)grid_for(chunk_encode<PER>, es, a.nc, num_sms);
+    a.per_range = (uint32_t)((a.nc + want - 1) / want);
+    a.ranges = a.nc ? (uint32_t)((a.nc + a.per_range - 1) / a.per_range) : 0u;
+    if (a.nc) chunk_encode<PER><<<a.ranges, kCT, es, stream>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    chunk_scan<<<1, kScanThreads, 0, stream>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.nc) chunk_gather<<<a.ranges, kCT, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -527,24 +587,12 @@ cudaError_t chunked_decode_as(const ChunkedDecArgs &a, uint64_t nc, int num_sms,
 uint64_t chunked_slot_words(uint32_t m) { return 1 + (uint64_t)((m + 31) & ~31u) + 2ull * m; }
 
 cudaError_t launch_chunked_encode(const ChunkedArgs &a, int num_sms, cudaStream_t stream) {
-    cudaError_t e;
     switch (a.m) {
-    case 1024: e = chunked_encode_as<4>(a, num_sms, stream); break;
-    case 2048: e = chunked_encode_as<8>(a, num_sms, stream); break;
-    case 4096: e = chunked_encode_as<16>(a, num_sms, stream); break;
+    case 1024: return chunked_encode_as<4>(a, num_sms, stream);
+    case 2048: return chunked_encode_as<8>(a, num_sms, stream);
+    case 4096: return chunked_encode_as<16>(a, num_sms, stream);
     default: return cudaErrorInvalidValue;
     }
-    if (e != cudaSuccess) return e;
-    chunk_scan<<<1, kScanThreads, 0, stream>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (a.nc) {
-        int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chunk_gather, kCT, 0) != cudaSuccess || per_sm < 1)
-            per_sm = 1;
-        const uint64_t want = (uint64_t)num_sms * per_sm;
-        chunk_gather<<<(int)(a.nc < want ? a.nc : want), kCT, 0, stream>>>(a);
-    }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_chunked_decode(const ChunkedDecArgs &a, int num_sms, cudaStream_t stream) {

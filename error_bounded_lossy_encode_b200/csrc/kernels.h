@@ -86,9 +86,10 @@ cudaError_t launch_decode(const DecodeArgs &a, int num_sms, cudaStream_t stream)
 
 // Chunk-cooperative codec (Quant -> Diff -> Bitshuffle -> RZE): chunks of m
 // = 1024, 2048 or 4096 elements.  One launch sequence writes the stream:
-// encode (each chunk's record into its scratch slot of chunked_slot_words(m)
-// words, its size and outlier count), scan (chunk index, header, result
-// block), gather (records to their offsets).
+// encode (CTA b codes the contiguous chunk range b: each chunk's record into
+// its scratch slot of chunked_slot_words(m) words, its size and outlier
+// count, the range's totals), scan (the ranges' bases, header, result
+// block), gather (per range: chunk index entries, records to their offsets).
 struct ChunkedArgs {
     const float *in;          // n floats
     uint64_t n;
@@ -99,7 +100,9 @@ struct ChunkedArgs {
     const float *range;       // vmin, vmax (relative mode)
     uint32_t *scratch;        // nc slots
     uint32_t slot_words;
-    uint32_t *sizes, *outl, *offs;  // nc each: record words, outliers, record word offset
+    uint32_t *sizes, *outl;   // nc each: record words, outliers
+    uint32_t *part;           // 2 nc: per chunk range, record words [0, nc) and outliers [nc, 2 nc)
+    uint32_t ranges, per_range;  // set by the launcher: chunk ranges, chunks per range
     uint8_t *out;
     uint64_t out_cap;
     uint64_t *result;         // as EncodeArgs::result

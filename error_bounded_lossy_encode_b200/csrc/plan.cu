@@ -356,7 +356,7 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
         ca.slot_words = (uint32_t)slot;
         ca.sizes = p->chunk_scratch ? p->chunk_scratch + p->L.nc * slot : nullptr;
         ca.outl = ca.sizes ? ca.sizes + p->L.nc : nullptr;
-        ca.offs = ca.outl ? ca.outl + p->L.nc : nullptr;
+        ca.part = ca.outl ? ca.outl + p->L.nc : nullptr;
         ca.out = d_out;
         ca.out_cap = cap;
         ca.result = p->d_rb->result;
@@ -635,8 +635,8 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
             base = static_cast<uint8_t *>(p->scratch);
         }
     }
-    if (p->chunked_m && p->L.nc) {  // record slots of the chunked codec, then sizes, outlier counts, offsets
-        const uint64_t words = p->L.nc * (chunked_slot_words(p->chunked_m) + 3);
+    if (p->chunked_m && p->L.nc) {  // record slots of the chunked codec, then sizes, outlier counts, range totals
+        const uint64_t words = p->L.nc * (chunked_slot_words(p->chunked_m) + 4);
         if ((s = cuda_status(cudaMalloc(&p->chunk_scratch, 4 * words), "cudaMalloc chunk scratch")) != EBLC_OK) {
             p->chunk_scratch = nullptr;
             destroy(p);
