@@ -194,13 +194,15 @@ __device__ __forceinline__ void tensor_g2s_2d(void *dst_smem, const void *tmap, 
 }
 
 // Brick t of a multi-dimensional array {Z, Y, X} in C order over the brick
-// grid: its first element's (z, y, x).
+// grid: its first element's (z, y, x).  Every dim and brick count is below
+// 2^30 (n <= 2^30), so 32-bit arithmetic is exact.
 __host__ __device__ inline void brick_origin(uint64_t t, int nd, const uint64_t *dims, int &z, int &y, int &x) {
-    const uint64_t ex = (nd == 3) ? 16 : 64, ey = ex, ez = (nd == 3) ? 16 : 1;
-    const uint64_t gx = dims[2] / ex, gy = dims[1] / ey;
-    x = (int)((t % gx) * ex);
-    y = (int)(((t / gx) % gy) * ey);
-    z = (int)((t / (gx * gy)) * ez);
+    const uint32_t ex = (nd == 3) ? 16u : 64u, ey = ex, ez = (nd == 3) ? 16u : 1u;
+    const uint32_t gx = (uint32_t)dims[2] / ex, gy = (uint32_t)dims[1] / ey, tt = (uint32_t)t;
+    const uint32_t ty = tt / gx;
+    x = (int)((tt - ty * gx) * ex);
+    y = (int)((ty % gy) * ey);
+    z = (int)((ty / gy) * ez);
 }
 
 __device__ __forceinline__ uint64_t ld_relaxed_gpu(const uint64_t *p) {

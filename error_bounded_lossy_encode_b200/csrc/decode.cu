@@ -104,9 +104,11 @@ __device__ __forceinline__ void widths_of_tile(const uint8_t *wb, int g, uint32_
 // 3-D 4x8x8 and 2-D 8x8 one row of 8; 2-D 16x16 half a row) summed back --
 // inclusive prefix sums along x, then y, then z within the block, by
 // segmented warp scans -- dequantized and stored at their places in the
-// array.  Brick t's block bi (C order within the brick).
+// array.  Block bi (C order within the brick) of the brick whose first
+// element is (bz, by, bx).
 template <int ND, int LPB>
-__device__ __forceinline__ void nd_store(const DecodeArgs &a, int tile, uint32_t bi, int r, const uint32_t (&d)[8]) {
+__device__ __forceinline__ void nd_store(const DecodeArgs &a, int bz, int by, int bx, uint32_t bi, int r,
+                                         const uint32_t (&d)[8]) {
     constexpr int kBX = (ND == 3) ? (LPB == 8 ? 4 : 8) : (LPB == 8 ? 8 : 16);
     constexpr int kBY = (ND == 3) ? (LPB == 8 ? 4 : 8) : (LPB == 8 ? 8 : 16);
     constexpr int kKX = ((ND == 3) ? 16 : 64) / kBX, kKY = ((ND == 3) ? 16 : 64) / kBY;
@@ -179,8 +181,6 @@ __device__ __forceinline__ void nd_store(const DecodeArgs &a, int tile, uint32_t
     float y[8];
 #pragma unroll
     for (int v = 0; v < 8; ++v) y[v] = __fmul_rn(__int2float_rn((int32_t)q[v]), a.step);
-    int bz, by, bx;
-    brick_origin((uint64_t)tile, ND, a.dims, bz, by, bx);
     const int kx = (int)(bi % kKX), ky = (int)((bi / kKX) % kKY), kz = (int)(bi / (kKX * kKY));
     const uint64_t z = (uint64_t)(bz + kz * ((ND == 3) ? 4 : 1) + zo);
     const uint64_t yy = (uint64_t)(by + ky * kBY + yo), x = (uint64_t)(bx + kx * kBX + xo);
@@ -214,6 +214,8 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
         const uint32_t *rec = sm.rec[s] + adj;
         const uint8_t *wid = sm.width[s];
         float *const gout = a.out + (uint64_t)tile * kChunk;
+        int bz = 0, by = 0, bx = 0;  // the brick's first element (multi-dimensional tiles)
+        if constexpr (ND != 0) brick_origin((uint64_t)tile, ND, a.dims, bz, by, bx);
 
         // widths of the chunk's blocks before this warp's first block
         const uint32_t blk0 = (uint32_t)(cw * kWPW * kWT) / kB;
@@ -303,7 +305,7 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
                     }
                 }
                 if constexpr (ND != 0) {
-                    nd_store<ND, LPB>(a, tile, (uint32_t)(wt * kWT) / kB + g, r, dv);
+                    nd_store<ND, LPB>(a, bz, by, bx, (uint32_t)(wt * kWT) / kB + g, r, dv);
                     before += tot;
                     continue;
                 }
@@ -353,14 +355,12 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
             for (uint32_t k = tid; k < mt; k += kNW * 32) {
                 const uint32_t idx = staged ? rec[PW + k] : gidx[k];
                 const uint32_t val = staged ? rec[PW + mt + k] : gidx[mt + k];
-                if constexpr (ND != 0) {  // the index must lie in this brick
-                    int bz, by, bx;
-                    brick_origin((uint64_t)tile, ND, a.dims, bz, by, bx);
-                    const uint64_t xx = idx % a.dims[2], yy = (idx / a.dims[2]) % a.dims[1];
-                    const uint64_t zz = idx / (a.dims[2] * a.dims[1]);
-                    const uint64_t ez = (ND == 3) ? 16 : 1, exy = (ND == 3) ? 16 : 64;
-                    if (idx < a.n && zz >= (uint64_t)bz && zz < bz + ez && yy >= (uint64_t)by && yy < by + exy &&
-                        xx >= (uint64_t)bx && xx < bx + exy)
+                if constexpr (ND != 0) {  // the index must lie in this brick (32-bit: n <= 2^30)
+                    const uint32_t X = (uint32_t)a.dims[2], Y = (uint32_t)a.dims[1];
+                    const uint32_t row = idx / X, xx = idx - row * X, zz = row / Y, yy = row - zz * Y;
+                    const uint32_t ez = (ND == 3) ? 16 : 1, exy = (ND == 3) ? 16 : 64;
+                    if (idx < a.n && zz >= (uint32_t)bz && zz < bz + ez && yy >= (uint32_t)by && yy < by + exy &&
+                        xx >= (uint32_t)bx && xx < bx + exy)
                         a.out[idx] = __uint_as_float(val);
                     else
                         atomicOr(a.err, kErrCorrupt);
