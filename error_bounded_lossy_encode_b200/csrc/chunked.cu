@@ -372,10 +372,24 @@ __global__ void __launch_bounds__(kCT) chunk_gather(const ChunkedArgs a) {
         __syncthreads();
         const uint32_t nw = (uint32_t)min((uint64_t)kCT, ce - c0);
         for (uint32_t k = w; k < nw; k += kCW) {
-            const uint64_t o = off_s[k], len = len_s[k];
+            const uint64_t o = off_s[k];
+            const uint32_t len = len_s[k];
             if (o + len > cap_words) continue;  // reported by chunk_scan (capacity)
             const uint32_t *src = a.scratch + (c0 + k) * (uint64_t)a.slot_words;
-            for (uint32_t j = ln; j < len; j += 32) st_cs_u32(recs + o + j, src[j]);
+            // eight loads in flight per lane before their stores
+            for (uint32_t j0 = 0; j0 < len; j0 += 8 * 32) {
+                uint32_t v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t j = j0 + 32 * u + ln;
+                    v[u] = (j < len) ? __ldg(src + j) : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t j = j0 + 32 * u + ln;
+                    if (j < len) st_cs_u32(recs + o + j, v[u]);
+                }
+            }
         }
         base_r += tr;
         base_m += tm;
