@@ -823,6 +823,63 @@ __device__ __forceinline__ void write_tile(EncSmem &sm, const EncodeArgs &a, con
     if (__any_sync(kFull, over) && ln == 0) atomicOr(a.err, kErrCapacity);
 }
 
+constexpr uint32_t kHeavySlice = 16;  // outliers in a slice from which write_slice_heavy takes it
+
+// One compute warp's slice of a full tile with many outliers (write_tile_fast
+// below takes the others): the lanes that have outliers reload their inputs
+// for both warp-tiles first, so those L2 round trips overlap the payload copy,
+// then the ranked outlier stores.  Kept out of line so that the common path's
+// code is not shaped by it.
+template <int V>
+__device__ __noinline__ void write_slice_heavy(const uint32_t *src, uint32_t *dst, uint32_t words, uint32_t om,
+                                               uint32_t *recs, uint32_t ord, uint32_t MT, const float *xin,
+                                               uint32_t i_tile, int c, int ln) {
+    constexpr int kWT = 32 * V;
+    constexpr int kWPW = kChunk / kWT / kNW;
+    float4 xr[kWPW][2];
+#pragma unroll
+    for (int k = 0; k < kWPW; ++k) {
+        const uint32_t e_loc = (uint32_t)(c * kWPW + k) * kWT + ln * V;
+        if ((om >> (k * V)) & ((1u << V) - 1u)) {
+            xr[k][0] = __ldg(reinterpret_cast<const float4 *>(xin + e_loc));
+            xr[k][1] = __ldg(reinterpret_cast<const float4 *>(xin + e_loc + 4));
+        }
+    }
+    uint32_t j = ln;
+    for (; j + 32 < words; j += 64) {
+        const uint32_t v0 = src[j], v1 = src[j + 32];
+        st_cs_u32(dst + j, v0);
+        st_cs_u32(dst + j + 32, v1);
+    }
+    if (j < words) st_cs_u32(dst + j, src[j]);
+#pragma unroll
+    for (int k = 0; k < kWPW; ++k) {
+        const uint32_t bits = (om >> (k * V)) & ((1u << V) - 1u);
+        const uint32_t cnt = __popc(bits);
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t t = __shfl_up_sync(kFull, incl, o);
+            if (ln >= o) incl += t;
+        }
+        if (bits != 0u) {
+            const float xv[V] = {xr[k][0].x, xr[k][0].y, xr[k][0].z, xr[k][0].w,
+                                 xr[k][1].x, xr[k][1].y, xr[k][1].z, xr[k][1].w};
+            uint32_t p = ord + incl - cnt;
+            const uint32_t i0 = i_tile + (uint32_t)(c * kWPW + k) * kWT + ln * V;
+#pragma unroll
+            for (int v = 0; v < V; ++v) {
+                if ((bits >> v) & 1u) {
+                    recs[p] = i0 + v;
+                    recs[p + MT] = __float_as_uint(xv[v]);
+                    ++p;
+                }
+            }
+        }
+        ord += __shfl_sync(kFull, incl, 31);
+    }
+}
+
 // write_tile for a full tile whose whole record (and its width bytes) fits
 // in the caller's capacity, checked once by the caller: no per-store checks.
 // Outliers: per warp-tile of a compute warp's slice, one warp scan of the
@@ -844,6 +901,11 @@ __device__ __forceinline__ void write_tile_fast(EncSmem &sm, const EncodeArgs &a
         const uint32_t words = sm.totals[q][c][0], pos = sm.ringpos[q][c], mc = sm.totals[q][c][1];
         const uint32_t *src = sm.ring[c] + pos;
         uint32_t *dst = recs + (rec + __shfl_sync(kFull, wpw, c));
+        if (mc >= kHeavySlice) {
+            write_slice_heavy<V>(src, dst, words, sm.omask[q][c][ln], recs, rec + PW + __shfl_sync(kFull, wpo, c),
+                                 MT, xin, (uint32_t)tile * kChunk, c, ln);
+            continue;
+        }
         uint32_t j = ln;
         for (; j + 32 < words; j += 64) {
             const uint32_t v0 = src[j], v1 = src[j + 32];
