@@ -88,7 +88,7 @@ struct eblc_plan_s {
     uint32_t chunked_m = 0;         // option codec=chunked: elements per chunk (1024, 2048, 4096), else 0
     int opt_chunked = 0;            // options as parsed (resolved by plan_create)
     uint32_t opt_chunk_bytes = 0;
-    uint32_t *chunk_scratch = nullptr;  // codec=chunked: nc record slots, then sizes, outlier counts, offsets
+    uint32_t *chunk_scratch = nullptr;  // codec=chunked: nc record slots, then sizes, outlier counts, range totals
     uint64_t dims[3] = {0, 0, 0};   // {Z, Y, X} of a multi-dimensional plan (Z = 1 for 2-D)
     uint64_t stall_call = 0;        // the compress call (0-based) that stall_tile applies to
     uint64_t calls = 0;             // compress calls enqueued so far

@@ -6,10 +6,12 @@
 // produced.  This is the compulsory first read of the input in relative mode.
 //
 // HBM-bound: 4 bytes read per element, no writes.  Persistent grid of one
-// wave of 256-thread CTAs; each thread keeps 8 float4 loads in flight
-// (fetched with a 256-byte L2 prefetch hint).
+// wave of 256-thread CTAs; each thread keeps 16 float4 loads in flight.
 // The array is walked from its end to its start so the lowest addresses are
-// the last read and are still in L2 when the encoder starts at tile 0.
+// the last read and are still in L2 when the encoder starts at tile 0: the
+// lowest kKeep4 float4 (48 MiB) are loaded with the normal L2 policy and a
+// 256-byte L2 prefetch hint, everything above with evict-first streaming
+// loads, so the streamed part does not push the kept part out of L2.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -17,7 +19,8 @@ namespace eblc {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kUnroll = 8;
+constexpr int kUnroll = 16;
+constexpr uint64_t kKeep4 = 3ull << 20;  // float4 at the array's start kept in L2 for the encoder
 
 __device__ __forceinline__ void fold(float v, float &lo, float &hi) {
     // +-Inf become NaN, which fminf / fmaxf ignore (as they ignore NaN itself)
@@ -46,7 +49,8 @@ __global__ void __launch_bounds__(kThreads) range_kernel(RangeArgs a) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const uint64_t i = base + u * stride + tid;
-            v[u] = (i < n4) ? ld_nc_256(in4 + (n4 - 1 - i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const uint64_t j = n4 - 1 - i;
+            v[u] = (i < n4) ? ((j < kKeep4) ? ld_nc_256(in4 + j) : __ldcs(in4 + j)) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
@@ -119,7 +123,7 @@ __global__ void __launch_bounds__(kThreads) range_kernel(RangeArgs a) {
 }  // namespace
 
 // One wave of resident CTAs (occupancy is set by the registers of the
-// 8-deep load unroll), at most 8 per SM.
+// 16-deep load unroll), at most 8 per SM.
 int range_grid(int num_sms) {
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, range_kernel, kThreads, 0) != cudaSuccess ||
