@@ -228,11 +228,10 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
             for (int k = 0; k < kWPW; ++k) {
                 const int wt = cw * kWPW + k;
                 const uint32_t e0 = wt * kWT + ln * V;
-                const uint32_t blk = (uint32_t)(wt * kWT) / kB + g;
                 uint32_t w, pre, tot;
-                bool over;
+                bool over;  // widths above 32 are reported once per chunk, below
                 widths_of_tile<LPB>(wid + (uint32_t)(wt * kWT) / kB, g, w, pre, tot, over);
-                if (over && r == 0 && blk * kB < valid) atomicOr(a.err, kErrCorrupt);
+                (void)over;
                 // bit position of this lane's first code in the chunk payload
                 const uint32_t bit0 = 32u * kEPL * (before + pre) + (uint32_t)r * V * w;
                 const uint32_t mask = (w == 32u) ? kFull : ((1u << w) - 1u);
@@ -242,13 +241,17 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
                 // The lane's codes occupy bits [bit0, bit0 + 8w) of the staged
                 // payload.  For narrow blocks the lane loads the few words that
                 // hold them once and shifts the codes out of registers; wider
-                // blocks read two words per code.  Every word read lies in the
-                // staged record (widths checked above): one test per lane.
+                // blocks read two words per code.  Every word index is clamped
+                // into the stage (lim words from rec): a valid stream's codes
+                // lie in its payload, far below the clamp, so it never acts;
+                // a corrupt stream's widths can only make the lane read other
+                // words of the stage, and the per-chunk payload check below
+                // reports it.
                 const uint32_t wmax = __reduce_max_sync(kFull, w);
-                const uint32_t wd0 = bit0 >> 5, sh0 = bit0 & 31u;
-                const bool inside = ((bit0 + V * w) >> 5) + 1 < kRecWords - adj;
-                if (wmax <= 8u && __all_sync(kFull, wd0 + 2 < kRecWords - adj)) {
+                const uint32_t lim = kRecWords - adj, sh0 = bit0 & 31u;
+                if (wmax <= 8u) {
                     static_assert(V == 8, "narrow path: 8 codes of <= 8 bits fit in 64 bits");
+                    const uint32_t wd0 = min(bit0 >> 5, lim - 3u);
                     uint32_t lo = __funnelshift_r(rec[wd0], rec[wd0 + 1], sh0);
                     uint32_t hi = __funnelshift_r(rec[wd0 + 1], rec[wd0 + 2], sh0);
 #pragma unroll
@@ -261,8 +264,9 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
                         run += d;
                         c[v] = (int32_t)run;
                     }
-                } else if (wmax <= 16u && __all_sync(kFull, wd0 + 4 < kRecWords - adj)) {
+                } else if (wmax <= 16u) {
                     // 8 codes of <= 16 bits: 128 bits, shifted out of four words
+                    const uint32_t wd0 = min(bit0 >> 5, lim - 5u);
                     uint32_t g0 = __funnelshift_r(rec[wd0], rec[wd0 + 1], sh0);
                     uint32_t g1 = __funnelshift_r(rec[wd0 + 1], rec[wd0 + 2], sh0);
                     uint32_t g2 = __funnelshift_r(rec[wd0 + 2], rec[wd0 + 3], sh0);
@@ -279,25 +283,12 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
                         run += d;
                         c[v] = (int32_t)run;
                     }
-                } else if (__all_sync(kFull, inside)) {
-#pragma unroll
-                    for (int v = 0; v < V; ++v) {
-                        const uint32_t b = bit0 + v * w;
-                        const uint32_t wd = b >> 5;
-                        const uint32_t zz = __funnelshift_r(rec[wd], rec[wd + 1], b & 31u) & mask;
-                        const uint32_t d = (zz >> 1) ^ (0u - (zz & 1u));  // inverse zigzag
-                        dv[v] = d;
-                        run += d;
-                        c[v] = (int32_t)run;
-                    }
                 } else {
 #pragma unroll
                     for (int v = 0; v < V; ++v) {
                         const uint32_t b = bit0 + v * w;
-                        const uint32_t wd = b >> 5;
-                        const uint32_t zz = (wd + 1 < kRecWords - adj)
-                                                ? (__funnelshift_r(rec[wd], rec[wd + 1], b & 31u) & mask)
-                                                : 0u;
+                        const uint32_t wd = min(b >> 5, lim - 2u);
+                        const uint32_t zz = __funnelshift_r(rec[wd], rec[wd + 1], b & 31u) & mask;
                         const uint32_t d = (zz >> 1) ^ (0u - (zz & 1u));  // inverse zigzag
                         dv[v] = d;
                         run += d;
@@ -327,15 +318,21 @@ __device__ void compute_warp(DecSmem &sm, const DecodeArgs &a, int cw, int ln) {
                 }
                 before += tot;
             }
-            // the chunk's payload must hold exactly the words its widths call for
+            // the chunk's widths must be at most 32, and its payload must hold
+            // exactly the words they call for
             if (cw == kNW - 1) {
                 const uint32_t nblk = (valid + kB - 1) / kB;
-                uint32_t sum = 0;
-                for (uint32_t b = ln; b + 1 < nblk; b += 32) sum += min((uint32_t)wid[b], 32u);
+                uint32_t sum = 0, wbig = 0;
+                for (uint32_t b = ln; b + 1 < nblk; b += 32) {
+                    sum += min((uint32_t)wid[b], 32u);
+                    wbig = max(wbig, (uint32_t)wid[b]);
+                }
                 sum = __reduce_add_sync(kFull, sum);
                 const uint32_t last_cnt = valid - (nblk - 1) * kB;
                 const uint32_t wl = min((uint32_t)wid[nblk - 1], 32u);
-                if (ln == 0 && kEPL * sum + (wl * last_cnt + 31u) / 32u != PW) atomicOr(a.err, kErrCorrupt);
+                const bool too_wide = __any_sync(kFull, wbig > 32u) || wid[nblk - 1] > 32u;
+                if (ln == 0 && (too_wide || kEPL * sum + (wl * last_cnt + 31u) / 32u != PW))
+                    atomicOr(a.err, kErrCorrupt);
             }
         }
 

@@ -63,6 +63,12 @@ def test_corrupt_streams(torch_cuda, orc):
         bad[128 + 3] = 40  # a width above 32: detected on the device
         st, chk, _ = g.decompress_np(bad, None)
         assert st == 0 and chk == E.EBLC_CORRUPT
+        nb = -(-x.size // 64)
+        for blk in (nb - 1, 64 * 3 + 17):  # the last block of the stream; one inside a later chunk
+            bad = s.copy()
+            bad[128 + blk] = 33
+            st, chk, _ = g.decompress_np(bad, None)
+            assert st == 0 and chk == E.EBLC_CORRUPT, blk
         bad = s.copy()
         off = SC.sections(h)
         bad[off["index"] + 8: off["index"] + 12] = np.frombuffer(np.uint32(0xFFFFFF).tobytes(), np.uint8)
