@@ -48,7 +48,7 @@ namespace {
 constexpr int kNW = 8;                    // compute warps
 constexpr int kS = 3;                     // input stages
 #ifndef EBLC_ENC_SLOTS
-#define EBLC_ENC_SLOTS 16
+#define EBLC_ENC_SLOTS 12
 #endif
 constexpr int kD = EBLC_ENC_SLOTS;        // tile slots: at most kD - 1 tiles computed but not finished
 #ifndef EBLC_ENC_LB
@@ -58,13 +58,16 @@ constexpr int kLookbackWarps = EBLC_ENC_LB;  // look-back and write-out warps
 constexpr int kProducerWarp = kNW + kLookbackWarps;
 constexpr int kThreads = (kNW + kLookbackWarps + 1) * 32;
 constexpr int kWindow = 10;               // look-back rows of 32 status words per round trip
-constexpr uint32_t kRing = 1536;          // packed words a compute warp can hold (3 worst-case tiles)
+constexpr uint32_t kRing = 1760;          // packed words a compute warp can hold (the rest of the CTA's shared memory)
 constexpr uint32_t kWarpMax = kChunk / kNW;  // most words a warp packs for one tile
 // A compute warp short of ring room waits only for the write-out of its own
 // earlier tiles, whose look-backs wait only for lower tiles: no cycle.  The
 // ring holds several typical tiles per warp so the compute warps can run
 // ahead of the look-back (kRing >= 2 kWarpMax lets a worst-case tile follow a
-// pending one without waiting).
+// pending one without waiting).  A warp starts a tile only with kWarpMax
+// contiguous free words, so the ring's size sets how many wide tiles can
+// wait for their write-out; it takes what two CTAs per SM leave after the
+// input stages and the 12 slots' bookkeeping.
 static_assert(kRing >= 2 * kWarpMax, "a worst-case part must fit beside a pending one");
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr uint64_t kInclBit = 1ull << 63;
