@@ -120,6 +120,12 @@ def lib():
         L.orc_max_chunked_bytes.restype = u64
         L.orc_compress_chunked.argtypes = [P, u64, u32, ctypes.c_int, dbl, u64, P, u64]
         L.orc_compress_chunked.restype = ctypes.c_int64
+        L.orc_compress_chunked_coder.argtypes = [P, u64, u32, ctypes.c_int, ctypes.c_int, dbl, u64, P, u64]
+        L.orc_compress_chunked_coder.restype = ctypes.c_int64
+        L.orc_rre.argtypes = [P, u32, P]
+        L.orc_rre.restype = u32
+        L.orc_unrre.argtypes = [P, u64, u32, P]
+        L.orc_unrre.restype = ctypes.c_int64
         L.orc_decompress.argtypes = [P, u64, P, u64]
         L.orc_decompress.restype = ctypes.c_int
         L.orc_block_codes.argtypes = [P, u64, u32, flt, P, P]
@@ -399,14 +405,37 @@ def unrze(words, mp: int):
     return out[:mp], int(k)
 
 
+def rre(words) -> np.ndarray:
+    """Repetition elimination: bitmap words (bit j: word j differs from word
+    j - 1, word -1 being 0), then the words that differ."""
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    out = np.zeros(max(w.size + w.size // 32, 1), np.uint32)
+    k = lib().orc_rre(_ptr(w), w.size, _ptr(out))
+    return out[:k]
+
+
+def unrre(words, mp: int):
+    """Inverse of rre for mp words; returns (words, consumed) or raises."""
+    w = np.ascontiguousarray(words, dtype=np.uint32)
+    src = w if w.size else np.zeros(1, np.uint32)
+    out = np.zeros(max(mp, 1), np.uint32)
+    k = lib().orc_unrre(_ptr(src), w.size, mp, _ptr(out))
+    if k < 0:
+        raise OracleError(int(k))
+    return out[:mp], int(k)
+
+
 def max_chunked_bytes(n: int, chunk_bytes: int, outlier_cap: int | None = None) -> int:
     return int(lib().orc_max_chunked_bytes(n, chunk_bytes, n if outlier_cap is None else outlier_cap))
 
 
 def compress_chunked(x, chunk_bytes: int = 16384, *, rel: float | None = None, abs: float | None = None,
-                     outlier_cap: int | None = None):
-    """The chunk-cooperative codec (Quant -> Diff -> Bitshuffle -> RZE, see
-    orc_compress_chunked): the stream as a uint8 array."""
+                     outlier_cap: int | None = None, coder: str = "rze"):
+    """The chunk-cooperative codec (Quant -> Diff -> Bitshuffle -> RZE, or
+    RRE with coder="rre"; see orc_compress_chunked_coder): the stream as a
+    uint8 array."""
+    if coder not in ("rze", "rre"):
+        raise ValueError("coder is rze or rre")
     x = _f32(x).reshape(-1)
     if (rel is None) == (abs is None):
         raise ValueError("exactly one of rel / abs")
@@ -414,8 +443,8 @@ def compress_chunked(x, chunk_bytes: int = 16384, *, rel: float | None = None, a
     cap = x.size if outlier_cap is None else int(outlier_cap)
     need = max(max_chunked_bytes(x.size, chunk_bytes, cap), 1)
     out = np.zeros(need, np.uint8)
-    rc = lib().orc_compress_chunked(_ptr(x), x.size, chunk_bytes, int(abs_mode), float(abs if abs_mode else rel),
-                                    cap, _ptr(out), need)
+    rc = lib().orc_compress_chunked_coder(_ptr(x), x.size, chunk_bytes, int(coder == "rre"), int(abs_mode),
+                                          float(abs if abs_mode else rel), cap, _ptr(out), need)
     if rc < 0:
         raise OracleError(int(rc))
     return out[:rc].copy()

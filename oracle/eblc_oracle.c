@@ -82,6 +82,7 @@
 #define ORC_FLAG_ABS 1u
 #define ORC_FLAG_LORENZO_ND 2u    /* 2-D / 3-D Lorenzo over the array's own dims */
 #define ORC_FLAG_CHUNKED 4u       /* chunk-cooperative codec: Diff -> Bitshuffle -> RZE */
+#define ORC_FLAG_RRE 8u           /* with the chunked codec: RRE in place of RZE */
 
 /* error codes returned as negative values */
 #define ORC_ERR_ARG (-1)
@@ -663,6 +664,7 @@ int orc_parse_header(const uint8_t *s, uint64_t bytes, orc_header *h) {
     h->dims[0] = get_u64(s + 96);
     h->dims[1] = get_u64(s + 104);
     h->dims[2] = get_u64(s + 112);
+    if ((h->flags & ORC_FLAG_RRE) && !(h->flags & ORC_FLAG_CHUNKED)) return ORC_ERR_CORRUPT;  /* RRE codes chunks only */
     if (h->flags & ORC_FLAG_CHUNKED) {
         if (h->magic != ORC_MAGIC || h->version != ORC_VERSION || h->block != 0 ||
             (h->chunk != 1024 && h->chunk != 2048 && h->chunk != 4096) || (h->flags & ORC_FLAG_LORENZO_ND) ||
@@ -826,7 +828,13 @@ static int decompress_nd(const uint8_t *s, const orc_header *h, float *out) {
  *   - RZE (zero elimination): one bitmap bit per shuffled word (bit j of the
  *     bitmap: word j is not zero; mp/32 bitmap words, least significant bit
  *     first), then the nonzero words in order;
- *   - a chunk whose RZE form is not smaller than its mp shuffled words keeps
+ *   - RRE (repetition elimination), the coder chosen in place of RZE: one
+ *     bitmap bit per shuffled word (bit j: word j differs from word j - 1,
+ *     word -1 being 0), then the words that differ, in order; a word whose
+ *     bit is clear equals the word before it, so each word is the last kept
+ *     word at or before it (0 before the first).  RZE is RRE with every
+ *     predecessor taken as 0;
+ *   - a chunk whose coded form is not smaller than its mp shuffled words keeps
  *     the shuffled words verbatim, so a coded chunk never exceeds its input;
  *   - record of a chunk: one word P | raw << 31 (P payload words follow),
  *     the payload, then the chunk's outlier indices and values (ascending
@@ -881,6 +889,40 @@ int64_t orc_unrze(const uint32_t *in, uint64_t avail, uint32_t mp, uint32_t *out
     return (int64_t)k;
 }
 
+/* Repetition elimination of mp words (mp a multiple of 32): returns the
+ * words written to out (mp / 32 bitmap words, then the words that differ
+ * from their predecessor, the predecessor of word 0 being 0).              */
+uint32_t orc_rre(const uint32_t *in, uint32_t mp, uint32_t *out) {
+    uint32_t nbm = mp / 32, k = nbm;
+    for (uint32_t i = 0; i < nbm; ++i) out[i] = 0;
+    for (uint32_t j = 0; j < mp; ++j) {
+        uint32_t pred = j ? in[j - 1] : 0u;
+        if (in[j] != pred) {
+            out[j >> 5] |= 1u << (j & 31u);
+            out[k++] = in[j];
+        }
+    }
+    return k;
+}
+
+/* Inverse: from `avail` words at in, mp words to out (a clear bit repeats
+ * the word before).  Returns the words consumed, or -1 if the bitmap calls
+ * for more words than avail.                                               */
+int64_t orc_unrre(const uint32_t *in, uint64_t avail, uint32_t mp, uint32_t *out) {
+    uint32_t nbm = mp / 32;
+    if (avail < nbm) return -1;
+    uint64_t k = nbm;
+    uint32_t last = 0;
+    for (uint32_t j = 0; j < mp; ++j) {
+        if ((in[j / 32] >> (j % 32)) & 1u) {
+            if (k >= avail) return -1;
+            last = in[k++];
+        }
+        out[j] = last;
+    }
+    return (int64_t)k;
+}
+
 static int chunk_bytes_ok(uint32_t cb) { return cb == 4096 || cb == 8192 || cb == 16384; }
 
 uint64_t orc_max_chunked_bytes(uint64_t n, uint32_t chunk_bytes, uint64_t outlier_cap) {
@@ -889,9 +931,11 @@ uint64_t orc_max_chunked_bytes(uint64_t n, uint32_t chunk_bytes, uint64_t outlie
     return layout_of(0, nc, nc + n + 31 * nc, outlier_cap).total;
 }
 
-int64_t orc_compress_chunked(const float *x, uint64_t n, uint32_t chunk_bytes, int abs_mode, double bound,
-                             uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
+/* coder 0: RZE, 1: RRE. */
+int64_t orc_compress_chunked_coder(const float *x, uint64_t n, uint32_t chunk_bytes, int coder, int abs_mode,
+                                   double bound, uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
     if (!chunk_bytes_ok(chunk_bytes) || !(bound >= 0.0) || !isfinite(bound)) return ORC_ERR_ARG;
+    if (coder != 0 && coder != 1) return ORC_ERR_ARG;
     if (n > ORC_MAX_N) return ORC_ERR_ARG;
     if (fegetround() != FE_TONEAREST) return ORC_ERR_ARG;
     float vmin = 0.0f, vmax = 0.0f;
@@ -927,7 +971,7 @@ int64_t orc_compress_chunked(const float *x, uint64_t n, uint32_t chunk_bytes, i
             memset(out, 0, L.total);
             put_u32(out + 0, ORC_MAGIC);
             put_u16(out + 4, (uint16_t)ORC_VERSION);
-            put_u16(out + 6, (uint16_t)((abs_mode ? ORC_FLAG_ABS : 0u) | ORC_FLAG_CHUNKED));
+            put_u16(out + 6, (uint16_t)((abs_mode ? ORC_FLAG_ABS : 0u) | ORC_FLAG_CHUNKED | (coder ? ORC_FLAG_RRE : 0u)));
             put_u64(out + 8, n);
             put_u32(out + 16, 0);
             put_u32(out + 20, mc_max);
@@ -957,7 +1001,7 @@ int64_t orc_compress_chunked(const float *x, uint64_t n, uint32_t chunk_bytes, i
                 }
             }
             orc_bitshuffle(d, mp, sh);
-            uint32_t r = orc_rze(sh, mp, rz);
+            uint32_t r = coder ? orc_rre(sh, mp, rz) : orc_rze(sh, mp, rz);
             int raw = r >= mp;
             uint32_t P = raw ? mp : r;
             uint64_t mc = 0;
@@ -991,6 +1035,11 @@ int64_t orc_compress_chunked(const float *x, uint64_t n, uint32_t chunk_bytes, i
     return ORC_ERR_ARG; /* not reached */
 }
 
+int64_t orc_compress_chunked(const float *x, uint64_t n, uint32_t chunk_bytes, int abs_mode, double bound,
+                             uint64_t outlier_cap, uint8_t *out, uint64_t out_cap) {
+    return orc_compress_chunked_coder(x, n, chunk_bytes, 0, abs_mode, bound, outlier_cap, out, out_cap);
+}
+
 static int decompress_chunked(const uint8_t *s, const orc_header *h, float *out) {
     uint32_t rec_words[4096 + 129], sh[4096], d[4096];
     uint64_t R = h->W + 2 * h->m, W_seen = 0;
@@ -1010,7 +1059,8 @@ static int decompress_chunked(const uint8_t *s, const orc_header *h, float *out)
         if (raw) {
             if (P != mp) return ORC_ERR_CORRUPT;
             memcpy(sh, rec_words, 4 * mp);
-        } else if (orc_unrze(rec_words, P, mp, sh) != (int64_t)P) {
+        } else if (((h->flags & ORC_FLAG_RRE) ? orc_unrre(rec_words, P, mp, sh) : orc_unrze(rec_words, P, mp, sh)) !=
+                   (int64_t)P) {
             return ORC_ERR_CORRUPT;
         }
         orc_unbitshuffle(sh, mp, d);

@@ -5,6 +5,8 @@
   bit order) and single-bit placements; the inverse round-trips;
 * RZE against a NumPy nonzero mask (bitmap packed little-endian, then the
   nonzero words); the inverse round-trips and rejects a short payload;
+* RRE against a NumPy "differs from the word before" mask and a hand-worked
+  example; its inverse against a NumPy forward fill of the kept words;
 * every stream decoded end to end in NumPy (record words, zero elimination,
   the bit matrix, zigzag, cumulative sum per chunk), compared with the
   quantiser's codes, with the outlier list and the bound on every element;
@@ -69,6 +71,48 @@ def test_rze_vs_numpy(orc, density):
             orc.unrze(r[:-1], 1024)
 
 
+def _np_rre(words):
+    pred = np.concatenate([np.zeros(1, np.uint32), words[:-1]])
+    keep = words != pred
+    bm = np.packbits(keep.astype(np.uint8), bitorder="little").view("<u4").astype(np.uint32)
+    return np.concatenate([bm, words[keep]])
+
+
+def _np_unrre(pay, mp):
+    """Each word is the last kept word at or before it (0 before the first)."""
+    keep = np.unpackbits(pay[:mp // 32].view(np.uint8), bitorder="little")[:mp].astype(bool)
+    vals = np.concatenate([np.zeros(1, np.uint32), pay[mp // 32:]])
+    return vals[np.cumsum(keep)], int(keep.sum())
+
+
+def test_rre_hand_worked(orc):
+    # words 0 0 5 5 5 7 0 0 (then zeros): 5, 7 and 0 differ from their predecessors at 2, 5, 6
+    w = np.zeros(32, np.uint32)
+    w[2:5], w[5] = 5, 7
+    r = orc.rre(w)
+    assert list(r) == [(1 << 2) | (1 << 5) | (1 << 6), 5, 7, 0]
+    back, used = orc.unrre(r, 32)
+    assert used == 4 and np.array_equal(back, w)
+    # a run of one nonzero value costs one word, where zero elimination keeps all of them
+    v = np.full(64, 9, np.uint32)
+    assert list(orc.rre(v)) == [1, 0, 9] and orc.rze(v).size == 2 + 64
+
+
+@pytest.mark.parametrize("density", [0.0, 0.05, 0.5, 1.0])
+def test_rre_vs_numpy(orc, density):
+    rng = np.random.default_rng(7 + int(density * 100))
+    w = rng.integers(0, 4, size=1024, dtype=np.uint32)  # few distinct values: runs and repeats
+    w[rng.random(1024) >= density] = 0
+    r = orc.rre(w)
+    assert np.array_equal(r, _np_rre(w))
+    back, used = orc.unrre(r, 1024)
+    want, kept = _np_unrre(r, 1024)
+    assert used == r.size == 32 + kept and np.array_equal(back, w) and np.array_equal(want, w)
+    if r.size > 32:
+        with pytest.raises(orc.OracleError):
+            orc.unrre(r[:-1], 1024)
+
+
 def _np_decode(stream):
     """Independent decode of a chunked stream: codes (int64) and the outlier
     (index, bits) pairs."""
@@ -76,6 +120,7 @@ def _np_decode(stream):
     (magic, version, flags, n, block, chunk, eb, inv2eb, step, vmin, vmax, nb, nc, W, m, total, bound) = \
         struct.unpack_from("<IHHQIIdffffQQQQQd", bytes(s[:128]))
     assert magic == 0x434C4245 and flags & 4 and block == 0 and nb == 0 and total == s.size
+    rre = bool(flags & 8)
     index_off = 128
     record_off = index_off + -(-8 * nc // 16) * 16
     index = s[index_off:index_off + 8 * nc].view("<u4").reshape(-1, 2).astype(np.int64)
@@ -96,6 +141,9 @@ def _np_decode(stream):
         if raw:
             assert P == mp
             sh = pay
+        elif rre:
+            sh, kept = _np_unrre(pay, mp)
+            assert P == mp // 32 + kept and P < mp  # verbatim only when repetition elimination would not shrink
         else:
             bits = np.unpackbits(pay[:mp // 32].view(np.uint8), bitorder="little")[:mp].astype(bool)
             sh = np.zeros(mp, np.uint32)
@@ -110,7 +158,7 @@ def _np_decode(stream):
         words_seen += 1 + P
     assert words_seen == W
     cat = lambda a: np.concatenate(a) if a else np.zeros(0, np.int64)
-    return codes, cat(oidx), cat(oval), dict(eb=eb, inv2eb=inv2eb, step=step, n=n, m=m, raw=raws)
+    return codes, cat(oidx), cat(oval), dict(eb=eb, inv2eb=inv2eb, step=step, n=n, m=m, raw=raws, rre=rre)
 
 
 def _check(orc, x, s):
@@ -127,12 +175,35 @@ def _check(orc, x, s):
     return h
 
 
+@pytest.mark.parametrize("coder", ["rze", "rre"])
 @pytest.mark.parametrize("cb", CHUNK_BYTES)
 @pytest.mark.parametrize("bound", [("rel", 1e-3), ("rel", 1e-6), ("abs", 1e-7), ("abs", 0.0)])
-def test_chunked_stream_independent_decode(orc, cb, bound):
+def test_chunked_stream_independent_decode(orc, cb, bound, coder):
     x = np.concatenate([WL.with_spikes((8, 32, 64), 3, p_nonfinite=2e-3), WL.edge_mix(cb // 4 * 2 + 77, 5),
                         WL.sine_noise(5000, 2)])
-    _check(orc, x, orc.compress_chunked(x, cb, **{bound[0]: bound[1]}))
+    h = _check(orc, x, orc.compress_chunked(x, cb, coder=coder, **{bound[0]: bound[1]}))
+    assert h["rre"] == (coder == "rre")
+
+
+def test_rre_stream_shrinks_repeated_words(orc):
+    """A ramp with a constant step per element quantizes to codes with one
+    constant first difference: every group's plane words repeat the group
+    before, so RRE keeps a word per plane change where RZE keeps every
+    nonzero plane word.  On sparse differences (a ramp that steps every 64
+    elements) a nonzero word is followed by zeros and RRE keeps both, so
+    there RZE is the smaller one."""
+    ramp = (np.arange(1 << 14, dtype=np.float64) * 0.004).astype(np.float32)
+    a = orc.compress_chunked(ramp, 16384, abs=1e-3, coder="rze")
+    b = orc.compress_chunked(ramp, 16384, abs=1e-3, coder="rre")
+    _check(orc, ramp, a)
+    _check(orc, ramp, b)
+    assert b.size < a.size
+    steps = (np.arange(1 << 14, dtype=np.float64) // 64 * 0.01).astype(np.float32)
+    a = orc.compress_chunked(steps, 16384, abs=1e-3, coder="rze")
+    b = orc.compress_chunked(steps, 16384, abs=1e-3, coder="rre")
+    _check(orc, steps, a)
+    _check(orc, steps, b)
+    assert a.size < b.size
 
 
 @pytest.mark.parametrize("cb", CHUNK_BYTES)
@@ -140,9 +211,10 @@ def test_chunked_verbatim_and_sizes(orc, cb):
     rng = np.random.default_rng(cb)
     # differences of codes up to 2^29 fill every bit plane: zero elimination cannot shrink, the chunk stays verbatim
     noise = rng.uniform(-1e9, 1e9, 3 * cb // 4).astype(np.float32)
-    s = orc.compress_chunked(noise, cb, abs=1.0)
-    h = _check(orc, noise, s)
-    assert any(h["raw"]) and s.size <= orc.max_chunked_bytes(noise.size, cb)
+    for coder in ("rze", "rre"):
+        s = orc.compress_chunked(noise, cb, abs=1.0, coder=coder)
+        h = _check(orc, noise, s)
+        assert any(h["raw"]) and s.size <= orc.max_chunked_bytes(noise.size, cb)
     smooth = orc.compress_chunked(WL.sine_noise(3 * cb // 4, 1), cb, rel=1e-3)
     assert not any(_check(orc, WL.sine_noise(3 * cb // 4, 1), smooth)["raw"])
     for n in (0, 1, 31, 33, cb // 4 - 1, cb // 4, cb // 4 + 1):

@@ -40,6 +40,10 @@ MUTATIONS = [
     ("chunk Diff without reset", "int32_t prev = 0;  /* Diff: 0 before the chunk's first code */",
      "static int32_t prev = 0;  /* Diff: 0 before the chunk's first code */"),
     ("verbatim when larger", "int raw = r >= mp;", "int raw = r > mp + 1000000;"),
+    ("repetition predecessor of word 0", "uint32_t pred = j ? in[j - 1] : 0u;", "uint32_t pred = j ? in[j - 1] : in[0];"),
+    ("repetition inverse fills zeros", "        out[j] = last;",
+     "        out[j] = ((in[j / 32] >> (j % 32)) & 1u) ? last : 0u;"),
+    ("repetition coder flag", "(coder ? ORC_FLAG_RRE : 0u)", "(coder ? 0u : 0u)"),
 ]
 
 
