@@ -167,7 +167,7 @@ def workload_config(args, n, block, mode, bound, world):
     """The `config` both arms report for the same workload."""
     c = {"workload": args.workload if not args.elements else f"{args.workload}[:{n}]", "n": int(n)}
     if args.codec == "chunked":
-        c.update(codec="chunked", chunk_bytes=args.chunk)
+        c.update(codec="chunked", chunk_bytes=args.chunk, coder=args.coder)
     else:
         c["block"] = block
         if args.lorenzo == "nd":
@@ -190,7 +190,7 @@ def nd_dims(args):
 def variant_suffix(args) -> str:
     """'' for the default codec, else the codec's tag in profile file names."""
     if args.codec == "chunked":
-        return f"_chunked{args.chunk}"
+        return f"_chunked{args.chunk}" + ("_rre" if args.coder == "rre" else "")
     return "_nd" if args.lorenzo == "nd" else ""
 
 
@@ -212,9 +212,9 @@ def host_info():
     return {"cpu_model": model, "cores_available": cores}
 
 
-def options_string(block, mode, bound, timing=False, codec="block", chunk=16384, lorenzo="1d"):
+def options_string(block, mode, bound, timing=False, codec="block", chunk=16384, lorenzo="1d", coder="rze"):
     if codec == "chunked":
-        o = f"{mode}={bound!r},codec=chunked,chunk={chunk}"
+        o = f"{mode}={bound!r},codec=chunked,chunk={chunk},coder={coder}"
     else:
         o = f"{mode}={bound!r},block={block}" + (",lorenzo=nd" if lorenzo == "nd" else "")
     return o + (",timing=1" if timing else "")
@@ -256,7 +256,7 @@ def profiled_traffic(kernel: str, workload_name: str):
 # CPU oracle legs
 
 def cpu_oracle_sample(x, block, mode, bound, repeats=1, all_cores=False, elems=CPU_SAMPLE_ELEMS, codec="block",
-                      chunk=16384, dims=None):
+                      chunk=16384, dims=None, coder="rze"):
     """Time the CPU oracle (compress + decompress) on the first `elems`
     elements: the plain single-threaded oracle, or (all_cores) the OpenMP
     build of the same steps (block codec, 1-D Lorenzo).  With dims (lorenzo
@@ -268,7 +268,7 @@ def cpu_oracle_sample(x, block, mode, bound, repeats=1, all_cores=False, elems=C
         return None
     s = x[:elems]
     if codec == "chunked":
-        comp = lambda v, **b: oracle.compress_chunked(v, chunk, **b)
+        comp = lambda v, **b: oracle.compress_chunked(v, chunk, coder=coder, **b)
         decomp = oracle.decompress
     elif dims:
         slab = int(np.prod(dims[1:]))
@@ -293,7 +293,7 @@ def cpu_oracle_sample(x, block, mode, bound, repeats=1, all_cores=False, elems=C
     gbs = repeats * 4 * s.size / (t_c + t_d) / 1e9
     cores = oracle.omp_threads() if all_cores else 1
     what = f"the oracle's steps run over chunks with OpenMP on {cores} threads" if all_cores else \
-        "single-threaded plain C oracle" + (f", chunked codec ({chunk}-byte chunks)" if codec == "chunked" else
+        "single-threaded plain C oracle" + (f", chunked codec ({chunk}-byte chunks, {coder})" if codec == "chunked" else
                                             ", multi-dimensional Lorenzo" if dims else "")
     part = "the whole workload" if s.size == x.size else f"first {s.size} elements ({4 * s.size >> 20} MiB) of the workload"
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
@@ -308,7 +308,7 @@ REFERENCE_BUDGET_S = 150.0  # wall-time budget of the reference arm's timed step
 
 
 def oracle_kwargs(args) -> dict:
-    return {"codec": args.codec, "chunk": args.chunk,
+    return {"codec": args.codec, "chunk": args.chunk, "coder": args.coder,
             "dims": nd_dims(args) if args.codec == "block" and args.lorenzo == "nd" else None}
 
 
@@ -375,7 +375,7 @@ def run_ours(args):
     kw = oracle_kwargs(args)
     dims = list(kw["dims"]) if kw["dims"] else [n]
     st, plan = E.eblc_plan_create(dims, None, options_string(block, mode, bound, True, args.codec, args.chunk,
-                                                              args.lorenzo))
+                                                              args.lorenzo, args.coder))
     if st != E.EBLC_OK:
         raise RuntimeError("plan_create: " + E.STATUS_NAMES[st])
     _, lim = E.eblc_plan_get_limits(plan)
@@ -716,6 +716,8 @@ def main(argv=None):
                     help="block: the fused block codec (default); chunked: the chunk-cooperative codec")
     ap.add_argument("--chunk", type=int, choices=(4096, 8192, 16384), default=16384,
                     help="bytes of input per chunk of the chunked codec")
+    ap.add_argument("--coder", choices=("rze", "rre"), default="rze",
+                    help="zero elimination of the chunked codec: rze (default) or rre")
     ap.add_argument("--lorenzo", choices=("1d", "nd"), default="1d",
                     help="nd: the 2-D / 3-D Lorenzo predictor over the workload's own shape")
     ap.add_argument("--sharded", action="store_true",
@@ -723,6 +725,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.codec == "chunked" and args.lorenzo == "nd":
         ap.error("--lorenzo nd belongs to the block codec")
+    if args.coder != "rze" and args.codec != "chunked":
+        ap.error("--coder belongs to the chunked codec")
     if args.sharded and (args.codec != "block" or args.lorenzo != "1d"):
         ap.error("--sharded runs the block codec with the 1-D predictor")
     if args.impl == "reference":

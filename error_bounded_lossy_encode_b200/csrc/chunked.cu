@@ -138,7 +138,7 @@ __host__ __device__ constexpr size_t enc_smem_bytes(uint32_t m) { return 4ull * 
 // keeps them in registers from the load to the bit transpose; the input of
 // the CTA's next chunk is loaded as soon as the current chunk's codes are
 // formed, so its latency overlaps the rest.
-template <int PER>
+template <int PER, bool RRE>
 __global__ void __launch_bounds__(kCT, PER == 4 ? 6 : PER == 8 ? 4 : 3) chunk_encode(const ChunkedArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint32_t *const sw = reinterpret_cast<uint32_t *>(smem_raw);
@@ -210,8 +210,14 @@ __global__ void __launch_bounds__(kCT, PER == 4 ? 6 : PER == 8 ? 4 : 3) chunk_en
         // in flag word t (lower 16 bits; G <= kCT).  Both totals are <= 4096.
         const uint32_t per = ((G + kCW - 1) / kCW) * 32;
         const uint32_t k0 = min(w * per, mp), k1 = min(k0 + per, mp);
+        // a word is kept when it is not zero (RZE) / differs from the word
+        // before it, word -1 being 0 (RRE)
+        auto kept = [&](uint32_t k, uint32_t v) {
+            const uint32_t pv = (RRE && k) ? sw[phys(k - 1, lg)] : 0u;
+            return v != pv;
+        };
         uint32_t cntw = 0;
-        for (uint32_t k = k0 + ln; k < k1; k += 32) cntw += __popc(__ballot_sync(kFull, sw[phys(k, lg)] != 0u));
+        for (uint32_t k = k0 + ln; k < k1; k += 32) cntw += __popc(__ballot_sync(kFull, kept(k, sw[phys(k, lg)])));
         const uint32_t ow = (t < (int)G) ? __popc(oflag[t]) : 0u;
         uint32_t tot;
         const uint32_t pre = block_excl(((ln == 0 ? cntw : 0u) << 16) | ow, tmp, &tot);
@@ -226,9 +232,10 @@ __global__ void __launch_bounds__(kCT, PER == 4 ? 6 : PER == 8 ? 4 : 3) chunk_en
             uint32_t base = __shfl_sync(kFull, pre >> 16, 0);
             for (uint32_t k = k0 + ln; k < k1; k += 32) {
                 const uint32_t v = sw[phys(k, lg)];
-                const uint32_t bal = __ballot_sync(kFull, v != 0u);
+                const bool kp = kept(k, v);
+                const uint32_t bal = __ballot_sync(kFull, kp);
                 if (ln == 0) rec[1 + k / 32] = bal;  // bitmap word k / 32: bit l = word 32 (k/32) + l
-                if (v) rec[1 + G + base + __popc(bal & ((1u << ln) - 1u))] = v;
+                if (kp) rec[1 + G + base + __popc(bal & ((1u << ln) - 1u))] = v;
                 base += __popc(bal);
             }
         }
@@ -321,7 +328,7 @@ __global__ void __launch_bounds__(kScanThreads) chunk_scan(const ChunkedArgs a) 
     uint32_t h[32] = {};
     const uint64_t ebits = (uint64_t)__double_as_longlong(bd.eb), bbits = (uint64_t)__double_as_longlong(a.bound);
     h[0] = kMagic;
-    h[1] = kVersion | ((uint32_t)((a.abs_mode ? kFlagAbs : 0) | kFlagChunked) << 16);
+    h[1] = kVersion | ((uint32_t)((a.abs_mode ? kFlagAbs : 0) | kFlagChunked | (a.rre ? kFlagRre : 0)) << 16);
     h[2] = (uint32_t)a.n;
     h[3] = (uint32_t)(a.n >> 32);
     h[4] = 0;  // no blocks
@@ -407,7 +414,7 @@ __host__ __device__ constexpr size_t dec_smem_bytes(uint32_t m) { return 4ull * 
 // reconstructions go out as whole 128-byte lines.  Thread 0 loads the index
 // entries and the head word of the CTA's next chunk one chunk ahead; the
 // payload and the first kCT outliers of a chunk come in one round of loads.
-template <int PER>
+template <int PER, bool RRE>
 __global__ void __launch_bounds__(kCT, PER == 4 ? 5 : PER == 8 ? 4 : 3) chunk_decode(const ChunkedDecArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     uint32_t *const pl = reinterpret_cast<uint32_t *>(smem_raw);  // payload (RZE form)
@@ -507,7 +514,12 @@ __global__ void __launch_bounds__(kCT, PER == 4 ? 5 : PER == 8 ? 4 : 3) chunk_de
             for (uint32_t j = j0; j < j1; ++j) {
                 const uint32_t bw = pl[j];
                 uint32_t v = 0;
-                if ((bw >> ln) & 1u) {
+                if constexpr (RRE) {
+                    // each word is the last kept word at or before it (0 before the first)
+                    const uint32_t r = base + __popc(bw & (lt | (1u << ln)));
+                    const uint32_t idx = G + r - 1u;
+                    v = (r != 0u && idx < P) ? pl[idx] : 0u;
+                } else if ((bw >> ln) & 1u) {
                     const uint32_t idx = G + base + __popc(bw & lt);
                     v = (idx < P) ? pl[idx] : 0u;
                 }
@@ -571,15 +583,16 @@ int grid_for(K kernel, size_t smem, uint64_t nc, int num_sms) {
 }
 
 // One contiguous chunk range per CTA of one resident wave.
-template <int PER>
+template <int PER, bool RRE>
 cudaError_t chunked_encode_as(ChunkedArgs a, int num_sms, cudaStream_t stream) {
     const size_t es = enc_smem_bytes(a.m);
-    cudaError_t e = cudaFuncSetAttribute(chunk_encode<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)es);
+    cudaError_t e =
+        cudaFuncSetAttribute(chunk_encode<PER, RRE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)es);
     if (e != cudaSuccess) return e;
-    const uint64_t want = (uint64_t)grid_for(chunk_encode<PER>, es, a.nc, num_sms);
+    const uint64_t want = (uint64_t)grid_for(chunk_encode<PER, RRE>, es, a.nc, num_sms);
     a.per_range = (uint32_t)((a.nc + want - 1) / want);
     a.ranges = a.nc ? (uint32_t)((a.nc + a.per_range - 1) / a.per_range) : 0u;
-    if (a.nc) chunk_encode<PER><<<a.ranges, kCT, es, stream>>>(a);
+    if (a.nc) chunk_encode<PER, RRE><<<a.ranges, kCT, es, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     chunk_scan<<<1, kScanThreads, 0, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -587,12 +600,13 @@ cudaError_t chunked_encode_as(ChunkedArgs a, int num_sms, cudaStream_t stream) {
     return cudaGetLastError();
 }
 
-template <int PER>
+template <int PER, bool RRE>
 cudaError_t chunked_decode_as(const ChunkedDecArgs &a, uint64_t nc, int num_sms, cudaStream_t stream) {
     const size_t ds = dec_smem_bytes(a.m);
-    cudaError_t e = cudaFuncSetAttribute(chunk_decode<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ds);
+    cudaError_t e =
+        cudaFuncSetAttribute(chunk_decode<PER, RRE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ds);
     if (e != cudaSuccess) return e;
-    if (nc) chunk_decode<PER><<<grid_for(chunk_decode<PER>, ds, nc, num_sms), kCT, ds, stream>>>(a);
+    if (nc) chunk_decode<PER, RRE><<<grid_for(chunk_decode<PER, RRE>, ds, nc, num_sms), kCT, ds, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -601,20 +615,26 @@ cudaError_t chunked_decode_as(const ChunkedDecArgs &a, uint64_t nc, int num_sms,
 uint64_t chunked_slot_words(uint32_t m) { return 1 + (uint64_t)((m + 31) & ~31u) + 2ull * m; }
 
 cudaError_t launch_chunked_encode(const ChunkedArgs &a, int num_sms, cudaStream_t stream) {
-    switch (a.m) {
-    case 1024: return chunked_encode_as<4>(a, num_sms, stream);
-    case 2048: return chunked_encode_as<8>(a, num_sms, stream);
-    case 4096: return chunked_encode_as<16>(a, num_sms, stream);
+    switch (a.m * 2 + (a.rre ? 1 : 0)) {
+    case 2048: return chunked_encode_as<4, false>(a, num_sms, stream);
+    case 2049: return chunked_encode_as<4, true>(a, num_sms, stream);
+    case 4096: return chunked_encode_as<8, false>(a, num_sms, stream);
+    case 4097: return chunked_encode_as<8, true>(a, num_sms, stream);
+    case 8192: return chunked_encode_as<16, false>(a, num_sms, stream);
+    case 8193: return chunked_encode_as<16, true>(a, num_sms, stream);
     default: return cudaErrorInvalidValue;
     }
 }
 
 cudaError_t launch_chunked_decode(const ChunkedDecArgs &a, int num_sms, cudaStream_t stream) {
     const uint64_t nc = (a.n + a.m - 1) / a.m;
-    switch (a.m) {
-    case 1024: return chunked_decode_as<4>(a, nc, num_sms, stream);
-    case 2048: return chunked_decode_as<8>(a, nc, num_sms, stream);
-    case 4096: return chunked_decode_as<16>(a, nc, num_sms, stream);
+    switch (a.m * 2 + (a.rre ? 1 : 0)) {
+    case 2048: return chunked_decode_as<4, false>(a, nc, num_sms, stream);
+    case 2049: return chunked_decode_as<4, true>(a, nc, num_sms, stream);
+    case 4096: return chunked_decode_as<8, false>(a, nc, num_sms, stream);
+    case 4097: return chunked_decode_as<8, true>(a, nc, num_sms, stream);
+    case 8192: return chunked_decode_as<16, false>(a, nc, num_sms, stream);
+    case 8193: return chunked_decode_as<16, true>(a, nc, num_sms, stream);
     default: return cudaErrorInvalidValue;
     }
 }

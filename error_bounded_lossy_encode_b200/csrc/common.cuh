@@ -20,6 +20,7 @@ constexpr uint32_t kVersion = 1;
 constexpr uint16_t kFlagAbs = 1;
 constexpr uint16_t kFlagLorenzoNd = 2;  // 2-D / 3-D Lorenzo over the array's dims (bytes 96..119: Z, Y, X)
 constexpr uint16_t kFlagChunked = 4;    // chunk-cooperative codec (Diff -> Bitshuffle -> RZE), no block widths
+constexpr uint16_t kFlagRre = 8;        // with kFlagChunked: RRE (repetition elimination) in place of RZE
 constexpr uint64_t kMaxN = 1ull << 30;
 
 // Device error word bits.

@@ -102,6 +102,7 @@ struct ChunkedArgs {
     uint32_t slot_words;
     uint32_t *sizes, *outl;   // nc each: record words, outliers
     uint32_t *part;           // 2 nc: per chunk range, record words [0, nc) and outliers [nc, 2 nc)
+    int rre;                  // coder: 0 RZE, 1 RRE
     uint32_t ranges, per_range;  // set by the launcher: chunk ranges, chunks per range
     uint8_t *out;
     uint64_t out_cap;
@@ -120,6 +121,7 @@ struct ChunkedDecArgs {
     float step;
     float *out;
     uint32_t *err;
+    int rre;                  // coder: 0 RZE, 1 RRE
 };
 cudaError_t launch_chunked_decode(const ChunkedDecArgs &a, int num_sms, cudaStream_t stream);
 

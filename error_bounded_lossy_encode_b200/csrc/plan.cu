@@ -87,6 +87,8 @@ struct eblc_plan_s {
     int nd = 0;                     // option lorenzo=nd: 2 or 3 (the plan's rank), 0 for the 1-D path
     uint32_t chunked_m = 0;         // option codec=chunked: elements per chunk (1024, 2048, 4096), else 0
     int opt_chunked = 0;            // options as parsed (resolved by plan_create)
+    int opt_coder = -1;             // option coder=: -1 unset, 0 rze, 1 rre (codec=chunked only)
+    int chunked_rre = 0;            // codec=chunked with the RRE coder
     uint32_t opt_chunk_bytes = 0;
     uint32_t *chunk_scratch = nullptr;  // codec=chunked: nc record slots, then sizes, outlier counts, range totals
     uint64_t dims[3] = {0, 0, 0};   // {Z, Y, X} of a multi-dimensional plan (Z = 1 for 2-D)
@@ -205,6 +207,10 @@ eblc_status_t parse_options(const char *options, eblc_plan_s *p, bool *timing) {
         } else if (key == "codec") {
             if (val == "chunked") p->opt_chunked = 1;
             else if (val != "lorenzo") return EBLC_INVALID_ARG;
+        } else if (key == "coder") {  // zero elimination of the chunked codec: rze or rre
+            if (val == "rze") p->opt_coder = 0;
+            else if (val == "rre") p->opt_coder = 1;
+            else return EBLC_INVALID_ARG;
         } else if (key == "chunk") {  // bytes of float32 input per chunk of the chunked codec
             if (!parse_int(val, &iv)) return EBLC_INVALID_ARG;
             if (iv != 4096 && iv != 8192 && iv != 16384) return EBLC_UNSUPPORTED;
@@ -357,6 +363,7 @@ eblc_status_t enqueue_compress(eblc_plan_s *p, cudaStream_t st, const float *d_i
         ca.sizes = p->chunk_scratch ? p->chunk_scratch + p->L.nc * slot : nullptr;
         ca.outl = ca.sizes ? ca.sizes + p->L.nc : nullptr;
         ca.part = ca.outl ? ca.outl + p->L.nc : nullptr;
+        ca.rre = p->chunked_rre;
         ca.out = d_out;
         ca.out_cap = cap;
         ca.result = p->d_rb->result;
@@ -422,6 +429,7 @@ cudaError_t launch_plan_decode(const eblc_plan_s *p, const DecodeArgs &da, cudaS
     ca.step = da.step;
     ca.out = da.out;
     ca.err = da.err;
+    ca.rre = p->chunked_rre;
     return launch_chunked_decode(ca, p->num_sms, st);
 }
 
@@ -435,7 +443,7 @@ eblc_status_t finish_compress(eblc_plan_s *p, size_t *compressed_bytes, void *h_
         sc.magic = kMagic;
         sc.version = (uint16_t)kVersion;
         sc.flags = (uint16_t)((p->abs_mode ? kFlagAbs : 0) | (p->nd ? kFlagLorenzoNd : 0) |
-                              (p->chunked_m ? kFlagChunked : 0));
+                              (p->chunked_m ? kFlagChunked : 0) | (p->chunked_rre ? kFlagRre : 0));
         sc.block = p->block;
         sc.chunk = p->chunked_m ? p->chunked_m : kChunk;
         sc.n = p->n;
@@ -467,6 +475,7 @@ eblc_status_t check_stream(const eblc_plan_s *p, const eblc_sidecar_t &sc, size_
     if (sc.magic != kMagic || sc.version != kVersion) return EBLC_CORRUPT;
     if (sc.chunk != (p->chunked_m ? p->chunked_m : kChunk)) return p->chunked_m ? EBLC_INVALID_ARG : EBLC_CORRUPT;
     if (((sc.flags & kFlagChunked) != 0) != (p->chunked_m != 0)) return EBLC_INVALID_ARG;  // the plan's codec
+    if (((sc.flags & kFlagRre) != 0) != (p->chunked_rre != 0)) return EBLC_INVALID_ARG;     // and its coder
     if (sc.n != p->n || sc.block != p->block) return EBLC_INVALID_ARG;
     if (((sc.flags & kFlagLorenzoNd) != 0) != (p->nd != 0)) return EBLC_INVALID_ARG;  // the plan's predictor
     if (sc.payload_words > sc.n + 32 * p->L.nc || sc.n_outliers > sc.n) return EBLC_CORRUPT;
@@ -561,7 +570,7 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
         return s;
     }
     p->n = n;
-    if (p->opt_chunk_bytes && !p->opt_chunked) {  // chunk= belongs to codec=chunked
+    if ((p->opt_chunk_bytes || p->opt_coder >= 0) && !p->opt_chunked) {  // chunk= and coder= belong to codec=chunked
         delete p;
         return EBLC_INVALID_ARG;
     }
@@ -571,6 +580,7 @@ EBLC_API eblc_status_t eblc_plan_create(eblc_plan_t *out, int rank, const int64_
             return EBLC_UNSUPPORTED;
         }
         p->chunked_m = (p->opt_chunk_bytes ? p->opt_chunk_bytes : 16384) / 4;
+        p->chunked_rre = p->opt_coder == 1;
         p->block = 0;  // no blocks: the stream has no width bytes
     }
     if (p->nd) {  // multi-dimensional Lorenzo: rank 2 or 3, dims multiples of the brick, block 64 or 256

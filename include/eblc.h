@@ -112,7 +112,8 @@ typedef struct {
     uint16_t version;       /* stream version (1)                    */
     uint16_t flags;         /* bit0: absolute bound; bit1: 2-D / 3-D
                                Lorenzo (lorenzo=nd); bit2: chunked
-                               codec (codec=chunked)                 */
+                               codec (codec=chunked); bit3: its RRE
+                               coder (coder=rre)                     */
     uint32_t block;         /* B (0 for the chunked codec)           */
     uint32_t chunk;         /* elements per chunk: 4096, or the
                                chunked codec's 1024 / 2048 / 4096    */
@@ -176,6 +177,11 @@ EBLC_API const char *eblc_status_string(eblc_status_t status);
  *                    return EBLC_UNSUPPORTED for such plans.  ("Pipeline
  *                    specialization internals", Chunk-cooperative path.)
  *   chunk=<bytes>    4096 | 8192 | 16384 (default 16384), with codec=chunked
+ *   coder=rze|rre    with codec=chunked: zero elimination (default) or
+ *                    repetition elimination (a bitmap of the words that
+ *                    differ from the word before, the first word's
+ *                    predecessor being 0, then those words); a plan decodes
+ *                    only streams of its own coder (else EBLC_INVALID_ARG)
  *   timing=1         record per-kernel device times (eblc_plan_kernel_times)
  *   wait_ms=<t>      limit of device-side waits in milliseconds (default 2000)
  *   stall_tile=<t>   test hook: tile t of one compress call never publishes

@@ -71,6 +71,7 @@ class _Args:
     codec = "block"
     chunk = 16384
     lorenzo = "1d"
+    coder = "rze"
 
 
 def test_report_line_contract(monkeypatch):
@@ -139,8 +140,9 @@ def test_codec_variants_name_themselves():
         lorenzo = "nd"
 
     c = bench.workload_config(Ch, 1 << 20, 64, "rel", 1e-3, 1)
-    assert c["codec"] == "chunked" and c["chunk_bytes"] == 4096 and "block" not in c
-    assert bench.options_string(64, "rel", 1e-3, False, "chunked", 4096) == "rel=0.001,codec=chunked,chunk=4096"
+    assert c["codec"] == "chunked" and c["chunk_bytes"] == 4096 and c["coder"] == "rze" and "block" not in c
+    assert bench.options_string(64, "rel", 1e-3, False, "chunked", 4096) == \
+        "rel=0.001,codec=chunked,chunk=4096,coder=rze"
     d = bench.workload_config(Nd, 1 << 27, 64, "rel", 1e-3, 1)
     assert d["lorenzo"] == "nd" and d["dims"] == [512, 512, 512] and d["block"] == 64
     assert bench.options_string(64, "rel", 1e-3, False, "block", 16384, "nd") == "rel=0.001,block=64,lorenzo=nd"

@@ -1,8 +1,9 @@
 """The chunk-cooperative codec (plan option codec=chunked) on the GPU,
 through the C ABI: streams byte-identical to the oracle's
-orc_compress_chunked and reconstructions bit-identical to its decode, for
-4096/8192/16384-byte chunks, both bound modes, ragged and empty inputs,
-verbatim chunks, the HOST execution kind; corrupt streams are reported."""
+orc_compress_chunked_coder and reconstructions bit-identical to its decode,
+for both coders (RZE, RRE), 4096/8192/16384-byte chunks, both bound modes,
+ragged and empty inputs, verbatim chunks, the HOST execution kind; corrupt
+streams and streams of the other coder are reported."""
 import numpy as np
 import pytest
 
@@ -26,10 +27,10 @@ def _ex(torch):
     return E.cuda_exec(torch.cuda.current_stream().cuda_stream)
 
 
-def _run(torch, orc, x, cb, **bound):
+def _run(torch, orc, x, cb, coder="rze", **bound):
     mode, val = next(iter(bound.items()))
-    want = orc.compress_chunked(x, cb, **bound)
-    st, plan = E.eblc_plan_create([x.size], None, f"{mode}={val!r},codec=chunked,chunk={cb}")
+    want = orc.compress_chunked(x, cb, coder=coder, **bound)
+    st, plan = E.eblc_plan_create([x.size], None, f"{mode}={val!r},codec=chunked,chunk={cb},coder={coder}")
     assert st == E.EBLC_OK, E.STATUS_NAMES[st]
     try:
         _, lim = E.eblc_plan_get_limits(plan)
@@ -43,7 +44,8 @@ def _run(torch, orc, x, cb, **bound):
         got = out[:nb].cpu().numpy()
         diff = np.flatnonzero(got[:min(got.size, want.size)] != want[:min(got.size, want.size)])
         assert got.size == want.size and diff.size == 0, (got.size, want.size, diff[:1])
-        assert sc.flags & 4 and sc.chunk == cb // 4 and sc.total_bytes == want.size
+        assert sc.flags & 4 and bool(sc.flags & 8) == (coder == "rre")
+        assert sc.chunk == cb // 4 and sc.total_bytes == want.size
         y = torch.empty(max(x.size, 4), dtype=torch.float32, device="cuda")
         for side in (sc, None):
             y.fill_(7.0)
@@ -56,26 +58,32 @@ def _run(torch, orc, x, cb, **bound):
     return want
 
 
+@pytest.mark.parametrize("coder", ["rze", "rre"])
 @pytest.mark.parametrize("cb", CHUNK_BYTES)
 @pytest.mark.parametrize("bound", [{"rel": 1e-3}, {"rel": 1e-6}, {"abs": 1e-7}, {"abs": 0.0}])
-def test_chunked_parity(torch_cuda, orc, cb, bound):
+def test_chunked_parity(torch_cuda, orc, cb, bound, coder):
     x = np.concatenate([WL.with_spikes((8, 32, 64), 3, p_nonfinite=2e-3), WL.edge_mix(cb // 4 * 2 + 77, 5),
                         WL.sine_noise(5000, 2)])
-    _run(torch_cuda, orc, x, cb, **bound)
+    _run(torch_cuda, orc, x, cb, coder, **bound)
 
 
+@pytest.mark.parametrize("coder", ["rze", "rre"])
 @pytest.mark.parametrize("cb", CHUNK_BYTES)
 @pytest.mark.parametrize("n", [0, 1, 31, 33, 1023, 1024, 1025, 4097, 3 * 4096 + 5])
-def test_chunked_sizes(torch_cuda, orc, cb, n):
-    _run(torch_cuda, orc, WL.edge_mix(n, n + cb), cb, rel=1e-3)
+def test_chunked_sizes(torch_cuda, orc, cb, n, coder):
+    _run(torch_cuda, orc, WL.edge_mix(n, n + cb), cb, coder, rel=1e-3)
 
 
+@pytest.mark.parametrize("coder", ["rze", "rre"])
 @pytest.mark.parametrize("cb", CHUNK_BYTES)
-def test_chunked_verbatim_and_fields(torch_cuda, orc, cb):
+def test_chunked_verbatim_and_fields(torch_cuda, orc, cb, coder):
     rng = np.random.default_rng(cb)
-    _run(torch_cuda, orc, rng.uniform(-1e9, 1e9, 3 * cb // 4 + 100).astype(np.float32), cb, abs=1.0)
-    _run(torch_cuda, orc, WL.kfield((16, 32, 64), 1), cb, rel=1e-4)
-    _run(torch_cuda, orc, WL.noise_zero_ramp(65536, 4), cb, abs=1e-7)
+    _run(torch_cuda, orc, rng.uniform(-1e9, 1e9, 3 * cb // 4 + 100).astype(np.float32), cb, coder, abs=1.0)
+    _run(torch_cuda, orc, WL.kfield((16, 32, 64), 1), cb, coder, rel=1e-4)
+    _run(torch_cuda, orc, WL.noise_zero_ramp(65536, 4), cb, coder, abs=1e-7)
+    # a constant step per element: every group repeats the one before (RRE's case)
+    _run(torch_cuda, orc, (np.arange(3 * cb // 4 + 50, dtype=np.float64) * 0.004).astype(np.float32), cb, coder,
+         abs=1e-3)
 
 
 def test_chunked_host_kind_and_unsupported(torch_cuda, orc):
@@ -111,7 +119,17 @@ def test_chunked_host_kind_and_unsupported(torch_cuda, orc):
         assert st == E.EBLC_OK and E.eblc_check(plan, _ex(torch)) == E.EBLC_CORRUPT
     finally:
         E.eblc_plan_destroy(plan)
-    for opts in ("rel=1e-3,chunk=8192", "rel=1e-3,codec=bogus"):
+    # a stream of the other coder is not this plan's
+    rre = orc.compress_chunked(x, 8192, rel=1e-3, coder="rre")
+    st, plan = E.eblc_plan_create([x.size], None, "rel=1e-3,codec=chunked,chunk=8192")
+    try:
+        d = torch.from_numpy(rre).cuda()
+        y = torch.empty(x.size, device="cuda")
+        assert E.eblc_decompress(plan, _ex(torch), d.data_ptr(), rre.size, None, y.data_ptr()) == E.EBLC_INVALID_ARG
+    finally:
+        E.eblc_plan_destroy(plan)
+    for opts in ("rel=1e-3,chunk=8192", "rel=1e-3,codec=bogus", "rel=1e-3,coder=rre",
+                 "rel=1e-3,codec=chunked,coder=bogus"):
         st, p2 = E.eblc_plan_create([4096], None, opts)
         assert st == E.EBLC_INVALID_ARG and not p2
     st, p2 = E.eblc_plan_create([4096], None, "rel=1e-3,codec=chunked,chunk=2048")
