@@ -12,8 +12,9 @@
 //                 32 x 32 bit transpose of every group (lane b gets bit plane
 //                 b) by a shuffle butterfly, zero elimination (a bitmap of the
 //                 nonzero words by ballots, the nonzero words compacted warp
-//                 by warp after one block scan) or the shuffled words
-//                 verbatim when that is not smaller, then the chunk's
+//                 by warp after one block scan; with the RRE coder the words
+//                 that differ from the word before instead) or the shuffled
+//                 words verbatim when that is not smaller, then the chunk's
 //                 outliers in ascending order; the record goes to the chunk's
 //                 scratch slot, its size to sizes[], the range's totals to
 //                 part[].
@@ -23,7 +24,8 @@
 //                 scan from the range's base), records from scratch to their
 //                 place in the stream.
 //   chunk_decode  one CTA per chunk: zero elimination undone (each warp a
-//                 run of bitmap words, ranks by popcounts), the inverse
+//                 run of bitmap words, ranks by popcounts; RRE: each word is
+//                 the last kept word at or before it), the inverse
 //                 transpose, zigzag undone and the prefix sum in each warp's
 //                 registers, one block scan of the warps' totals,
 //                 dequantization, outliers.
